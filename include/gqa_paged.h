@@ -1,0 +1,196 @@
+/*
+ * gqa_paged.h -- C ABI of libgqa_paged.so: grouped-query attention (GQA) over a paged
+ * KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources by page title and section):
+ *   - GQA: Hq query heads form Hk groups of g = Hq/Hk consecutive heads; every head of a
+ *     group reads the same K/V head, kv head = h / g
+ *     ("TensorRT对Grouped Query Attention的支持进展", sections
+ *     "技术演进背景：从MHA到GQA的必然选择" and "图优化与算子融合", RepeatKV).
+ *   - Paged KV cache: each sequence's keys and values live in fixed-size pages of a pool
+ *     owned by the caller; a per-sequence page table maps logical page p to a physical
+ *     page ("TensorRT-LLM与TensorRT核心差异解析", section 4.2.2 PageAttention;
+ *     "TensorRT对Grouped Query Attention的支持进展", section "动态形状与KV Cache管理":
+ *     the caller keeps the pool and passes physical page indices on every call).
+ *   - Fused attention: softmax(scale * q K^T) V computed tile by tile on chip, only the
+ *     output written back ("TensorRT-LLM与TensorRT核心差异解析", section 4.2.1).
+ *   - PackGQA and NumSplits ("解锁GQA性能潜力：从批量大小敏感性到高效优化实践",
+ *     section "核心参数调优：PackGQA与NumSplits的协同舞蹈"): all query heads of a group
+ *     share one thread block so each KV page is read once; long contexts are split
+ *     across thread blocks and merged by log-sum-exp (lse_combine).
+ *   - Chunked prefill ("TensorRT对Grouped Query Attention的支持进展", section
+ *     "与动态批处理协同").
+ *   - FP8 KV ("解锁GQA性能潜力…", section "实践验证：从理论到落地的性能跃迁").
+ *
+ * Common conventions for every call:
+ *   - Every data pointer is a DEVICE pointer owned by the caller.  The library keeps
+ *     no reference after the call returns and allocates no device memory; scratch
+ *     space comes from the caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream).
+ *   - Return value: GQA_OK (0) when the work was enqueued; a negative gqa_status_t when
+ *     host-side validation failed (then nothing was enqueued) or a launch failed.
+ *   - Device-side errors (a page-table entry outside [0, num_pages), a bounded wait that
+ *     ran out) are recorded in an int32 error word at the start of `workspace` and read
+ *     and cleared by gqa_get_error().  A workspace must be zero-filled once before its
+ *     first use; after that the library only ever sets the word and gqa_get_error()
+ *     clears it.
+ *   - Layouts are row-major (C order).  KV pools are [num_pages][Hk][page_size][head_dim]
+ *     ("HND": each (page, kv head) block is one contiguous run).  q and out are bf16.
+ *   - Sequence lengths count the current token(s): the caller has already written the
+ *     new K/V into the cache.  The library never writes the cache.
+ *   - Page-table entries at or beyond ceil(seq_len / page_size) are never read; entries
+ *     may repeat across and within sequences (shared prefix pages).
+ *   - A sequence of length 0 yields output 0 and lse = -inf.
+ *   - The device arrays must not change until the enqueued work has finished.
+ */
+#ifndef GQA_PAGED_H_
+#define GQA_PAGED_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_NULL = -1,      /* a required pointer is NULL */
+    GQA_ERR_SHAPE = -2,     /* unsupported or inconsistent sizes (Hq % Hk, head_dim, page_size, ...) */
+    GQA_ERR_DTYPE = -3,     /* unknown kv_dtype, or fp8 without scales, or fp8 with head_dim != 128 */
+    GQA_ERR_SPLITS = -4,    /* num_splits outside 0..GQA_MAX_SPLITS */
+    GQA_ERR_WORKSPACE = -5, /* workspace NULL, smaller than the *_workspace_size() value, or not 256-byte aligned */
+    GQA_ERR_LAUNCH = -6,    /* a CUDA launch or driver call failed */
+    GQA_ERR_BAD_PAGE = -7,  /* (device) a page-table entry read was outside [0, num_pages) */
+    GQA_ERR_TIMEOUT = -8,   /* (device) a bounded pipeline wait ran out; the kernel gave up */
+    GQA_ERR_ALIGN = -9      /* a pointer is not 16-byte aligned */
+} gqa_status_t;
+
+typedef enum {
+    GQA_KV_BF16 = 0,     /* k_pages / v_pages hold bf16 */
+    GQA_KV_FP8_E4M3 = 1  /* k_pages / v_pages hold OCP e4m3 bytes; value = code * scale[page][kv head] */
+} gqa_kv_dtype_t;
+
+#define GQA_MAX_SPLITS 64
+
+/*
+ * Bytes of workspace gqa_paged_decode() needs for `num_splits` splits (0 = the value
+ * gqa_pick_splits() would choose for a context of up to max_seq_len tokens).  Layout:
+ * a 256-byte header holding the device error word, then, when the call splits,
+ * o_part fp32 [S][B*Hq][head_dim] and lse_part fp32 [S][B*Hq].
+ */
+size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int page_size,
+                                       int max_seq_len, int kv_dtype, int num_splits);
+
+/*
+ * Split count used when gqa_paged_decode() is called with num_splits = 0: a table
+ * measured on B200 over batch size B, kv heads Hk and the longest context (tokens).
+ */
+int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype);
+
+/*
+ * Decode: one new query token per sequence attends to all seq_lens[b] tokens of its
+ * paged history.  For sequence b and query head h (kv head j = h / (Hq/Hk)):
+ *   s_t = scale * <q[b][h], K_b[t]>,  out[b][h] = sum_t softmax(s)_t V_b[t],
+ *   lse[b][h] = ln sum_t exp(s_t)
+ * with K_b[t] = k_pages[page_table[b][t / page_size]][j][t % page_size].
+ *
+ *   q          bf16 [B][Hq][head_dim]
+ *   k_pages,
+ *   v_pages    [num_pages][Hk][page_size][head_dim] of kv_dtype; 16-byte aligned
+ *   k_scale,
+ *   v_scale    fp32 [num_pages][Hk] for GQA_KV_FP8_E4M3; ignored (may be NULL) for bf16
+ *   page_table int32 [B][pt_stride]; pt_stride >= ceil(max seq_len / page_size)
+ *   seq_lens   int32 [B], each in [0, pt_stride * page_size]
+ *   Hq % Hk == 0; head_dim in {64, 128}; page_size in {16, 32, 64}
+ *   scale      softmax scale (commonly 1/sqrt(head_dim))
+ *   num_splits 0 = automatic (gqa_pick_splits over max context pt_stride*page_size),
+ *              else 1..GQA_MAX_SPLITS contiguous page-aligned ranges of
+ *              ceil(np / num_splits) pages (np = ceil(seq_len / page_size)); the split
+ *              results are merged with lse_combine on the same stream
+ *   pack_gqa   1 (default): all heads of a group in one thread block, each KV page read
+ *              once; 0: one query head per thread block (for comparison sweeps only)
+ *   out        bf16 [B][Hq][head_dim]
+ *   lse        fp32 [B][Hq] natural-log log-sum-exp, or NULL
+ *   workspace  >= gqa_paged_decode_workspace_size(...) bytes, 256-byte aligned, zeroed
+ *              before first use
+ */
+int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
+                     const float *k_scale, const float *v_scale, int kv_dtype,
+                     const int32_t *page_table, int pt_stride, const int32_t *seq_lens, int B,
+                     int Hq, int Hk, int head_dim, int page_size, int num_pages, float scale,
+                     int num_splits, int pack_gqa, void *out, float *lse, void *workspace,
+                     size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Bytes of workspace gqa_paged_prefill() needs (the 256-byte error-word header).
+ */
+size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim);
+
+/*
+ * Causal chunked prefill: sequence b appends Lq_b = cu_q[b+1] - cu_q[b] new query tokens
+ * after a paged prior context; the chunk's K/V are already the last Lq_b of the
+ * seq_lens[b] cached tokens.  Query row i of sequence b sits at position
+ * pos = seq_lens[b] - Lq_b + i and, when causal, attends to tokens 0..pos (all
+ * seq_lens[b] tokens when causal == 0).
+ *
+ *   q          bf16 [total_q][Hq][head_dim], rows of sequence b at cu_q[b] .. cu_q[b+1]-1
+ *   cu_q       int32 [B+1], cu_q[0] = 0, nondecreasing, cu_q[B] = total_q,
+ *              cu_q[b+1] - cu_q[b] <= max_q_len and <= seq_lens[b]
+ *   k_pages, v_pages, page_table, pt_stride, seq_lens: as for decode (bf16 KV only)
+ *   head_dim   128; page_size in {16, 32, 64}
+ *   out        bf16 [total_q][Hq][head_dim];  lse fp32 [total_q][Hq] or NULL
+ *   workspace  >= gqa_paged_prefill_workspace_size(...) bytes, zeroed before first use
+ */
+int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
+                      const void *v_pages, const int32_t *page_table, int pt_stride,
+                      const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim,
+                      int page_size, int num_pages, float scale, int causal, int total_q,
+                      int max_q_len, void *out, float *lse, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Log-sum-exp merge of split attention results ("解锁GQA性能潜力…", NumSplits).  For
+ * every row r:  M = max_s lse_part[s][r],  w_s = exp(lse_part[s][r] - M),
+ *   out[r] = sum_s w_s o_part[s][r] / sum_s w_s,   lse[r] = M + ln sum_s w_s.
+ * Rows whose splits are all empty (lse = -inf) give out = 0, lse = -inf.
+ *
+ *   o_part   fp32 [num_splits][rows][head_dim], each split's output already normalised
+ *   lse_part fp32 [num_splits][rows], natural log
+ *   out      bf16 [rows][head_dim];  lse fp32 [rows] or NULL
+ *   1 <= num_splits <= GQA_MAX_SPLITS, head_dim in {64, 128}
+ */
+int lse_combine(const float *o_part, const float *lse_part, int num_splits, int rows,
+                int head_dim, void *out, float *lse, cudaStream_t stream);
+
+/*
+ * Copy-out of the paged cache into contiguous per-sequence storage, bit for bit:
+ *   k_out[cu_kv[b] + t][j][:] = k_pages[page_table[b][t / page_size]][j][t % page_size][:]
+ * and the same for v, for t < seq_lens[b].  elem_bytes is 2 (bf16) or 1 (fp8); bytes
+ * are copied, never interpreted.  A check of the page-table indirection on its own.
+ *
+ *   cu_kv    int64 [B+1] output row offsets (cu_kv[b+1] - cu_kv[b] = seq_lens[b])
+ *   k_out, v_out  [cu_kv[B]][Hk][head_dim] elements
+ * Page-table entries outside [0, num_pages) are not read; their rows are left unwritten
+ * and the call still succeeds (use the decode error word to detect bad tables).
+ */
+int gqa_paged_gather(const void *k_pages, const void *v_pages, const int32_t *page_table,
+                     int pt_stride, const int32_t *seq_lens, const int64_t *cu_kv, int B,
+                     int Hk, int head_dim, int page_size, int num_pages, int elem_bytes,
+                     void *k_out, void *v_out, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, returns the device error word held in `workspace`
+ * (GQA_OK or a negative gqa_status_t) and resets it to GQA_OK.
+ */
+int gqa_get_error(void *workspace, cudaStream_t stream);
+
+/* Human-readable name of a gqa_status_t value (static string). */
+const char *gqa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_PAGED_H_ */
