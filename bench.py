@@ -1,7 +1,432 @@
-"""Benchmark of paged GQA decode on B200 (placeholder: byte model only)."""
+"""Benchmark: paged GQA decode on B200 -- HBM GB/s (% of peak) and queries/s at B=64, 2K ctx.
 
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--B 64] [--ctx 2048] [--splits 0] [--no-pack] [--kv bf16|fp8_e4m3]
+
+One step = one gqa_paged_decode call (decode kernel + log-sum-exp merge when split) over
+a batch of B sequences, each with `ctx` tokens of paged history (Hq=32, Hk=8, D=128,
+page_size=16, seeded synthetic N(0,1) data).  Under torchrun every rank runs its own batch
+(weak scaling; no collective on the data path) and rank 0 prints one JSON line.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "GQA paged decode: HBM GB/s (% of B200 peak) and queries/s at B=64, 2K ctx"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------------ byte model
 
 def decode_kv_bytes(seq_lens, Hk, D, elem):
     """Algorithmic K+V bytes of one decode step: every valid token's K and V row of every
     kv head, read once."""
     return 2 * sum(int(L) for L in seq_lens) * Hk * D * elem
+
+
+def decode_step_bytes(seq_lens, Hq, Hk, D, elem, P=16):
+    """KV (read once) + q (bf16, read) + out (bf16, written); fp8 adds the per-(page, kv
+    head) K and V scales of every page read."""
+    B = len(seq_lens)
+    b = decode_kv_bytes(seq_lens, Hk, D, elem) + 2 * B * Hq * D * 2
+    if elem == 1:
+        b += 2 * 4 * Hk * sum((int(L) + P - 1) // P for L in seq_lens)
+    return b
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_src_sha():
+    h = hashlib.sha256()
+    for rel in ["gqa_attention_paged_b200/csrc/decode.cu", "gqa_attention_paged_b200/csrc/gqa_device.cuh",
+                "gqa_attention_paged_b200/csrc/combine.cu"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(workload_key):
+    """DRAM bytes per decode launch from the committed ncu summary, or None if absent or
+    taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_src_sha") != kernel_src_sha():
+        return None
+    e = d.get("workloads", {}).get(workload_key)
+    return None if e is None else float(e["dram_bytes_per_launch"])
+
+
+# ------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ CPU oracle leg
+
+def run_oracle_sample(case, rows, min_seconds):
+    """Time the fp64 oracle on sequences `rows` of `case`, repeating until min_seconds."""
+    import numpy as np
+    from oracle import oracle
+
+    kv = case.kv
+
+    def bits(t):
+        t = t.contiguous()
+        return t.view(__import__("torch").int16).numpy().view(np.uint16) if t.dtype.itemsize == 2 \
+            else t.view(__import__("torch").uint8).numpy()
+
+    q = bits(case.q[rows])
+    kp, vp = bits(kv.k_pages), bits(kv.v_pages)
+    pt = kv.page_table[rows].numpy()
+    sl = kv.seq_lens[rows].numpy()
+    ks = None if kv.k_scale is None else kv.k_scale.numpy()
+    vs = None if kv.v_scale is None else kv.v_scale.numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode(q, kp, vp, pt, sl, case.scale, ks, vs)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return el / reps, reps, oracle.num_threads()
+
+
+# ------------------------------------------------------------------------ main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--B", type=int, default=64)
+    ap.add_argument("--ctx", type=int, default=2048)
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-pack", action="store_true")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8_e4m3"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print one line per (B, splits, pack) point instead of the headline")
+    return ap.parse_args()
+
+
+def workload_name(a):
+    return (f"paged GQA decode, B={a.B} ctx={a.ctx} Hq=32 Hk=8 D=128 page_size=16 "
+            f"kv={a.kv}")
+
+
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        return reference_arm(a, world)
+
+    import torch
+    from gqa_attention_paged_b200 import binding, inputs
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    case = inputs.sweep_decode(a.B, seed=a.seed + rank, ctx=a.ctx, kv_dtype=a.kv)
+    kv = case.kv
+    q = case.q.to(dev)
+    kp, vp = kv.k_pages.to(dev), kv.v_pages.to(dev)
+    ks = None if kv.k_scale is None else kv.k_scale.to(dev)
+    vs = None if kv.v_scale is None else kv.v_scale.to(dev)
+    pt, sl = kv.page_table.to(dev), kv.seq_lens.to(dev)
+    elem = 1 if a.kv == "fp8_e4m3" else 2
+    B, Hq, Hk, D, P = a.B, 32, 8, 128, 16
+    kvc = binding.GQA_KV_FP8_E4M3 if elem == 1 else binding.GQA_KV_BF16
+    S = a.splits if a.splits > 0 else binding.gqa_pick_splits(B, Hk, pt.shape[1] * P, P, kvc)
+    pack = not a.no_pack
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ws = binding.new_workspace(
+        binding.gqa_paged_decode_workspace_size(B, Hq, Hk, D, P, pt.shape[1] * P, kvc, S), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.gqa_paged_decode(q, kp, vp, pt, sl, case.scale, num_splits=S, pack_gqa=pack,
+                                 k_scale=ks, v_scale=vs, out=out, lse=lse, workspace=ws,
+                                 stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # parity spot check of this exact launch configuration before timing
+    step()
+    torch.cuda.synchronize(dev)
+    assert binding.gqa_get_error(ws) == 0
+    assert torch.isfinite(out.float()).all(), "non-finite output"
+
+    for _ in range(max(3, a.warmup)):
+        step()
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(a.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    ms = ev0.elapsed_time(ev1) / a.steps
+    clk = clocks.stop()
+    ms = max_over_ranks(ms)
+
+    # The dominant kernel alone: time the merge kernel by itself on the same partials and
+    # subtract it (when the call splits), all with events on this stream.
+    comb_ms = 0.0
+    if S > 1:
+        hdr = 256
+        rows = B * Hq
+        o_bytes = (S * rows * D * 4 + 255) // 256 * 256
+        o_part = ws[hdr:hdr + S * rows * D * 4].view(torch.float32).view(S, rows, D)
+        l_part = ws[hdr + o_bytes:hdr + o_bytes + S * rows * 4].view(torch.float32).view(S, rows)
+        o2 = torch.empty(rows, D, dtype=torch.bfloat16, device=dev)
+        l2 = torch.empty(rows, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            binding.lse_combine(o_part, l_part, o2, l2, stream=stream)
+        torch.cuda.synchronize(dev)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(a.steps):
+            binding.lse_combine(o_part, l_part, o2, l2, stream=stream)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        comb_ms = c0.elapsed_time(c1) / a.steps
+    kern_ms = max(ms - comb_ms, 1e-6)
+
+    # end to end through the public API: per step, the step's inputs (q, page table,
+    # sequence lengths) copied from pinned host memory, the decode, and the result (out,
+    # lse) copied back; the KV cache is device-resident state.
+    hq = case.q.pin_memory()
+    hpt = kv.page_table.pin_memory()
+    hsl = kv.seq_lens.pin_memory()
+    hout = torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory()
+    hlse = torch.empty(B, Hq, dtype=torch.float32).pin_memory()
+    h2d = hq.numel() * 2 + hpt.numel() * 4 + hsl.numel() * 4
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        pt.copy_(hpt, non_blocking=True)
+        sl.copy_(hsl, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / a.steps)
+
+    lens = [int(x) for x in kv.seq_lens]
+    step_bytes = decode_step_bytes(lens, Hq, Hk, D, elem, P)
+    peak, peak_kind = peaks()
+    gbs = world * step_bytes / (ms * 1e-3) / 1e9
+    kern_gbs = step_bytes / (kern_ms * 1e-3) / 1e9
+    e2e_gbs = world * step_bytes / (e2e_ms * 1e-3) / 1e9
+    wkey = f"B{B}_ctx{a.ctx}_{a.kv}_S{S}_pack{int(pack)}"
+    traffic = traffic_from_profile(wkey)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rows = list(range(min(B, 8)))
+        sec, reps, cores = run_oracle_sample(case, rows, a.cpu_seconds)
+        sb = decode_step_bytes([lens[r] for r in rows], Hq, Hk, D, elem, P)
+        cpu = {"value": sb / sec / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{len(rows)} of {B} sequences (ctx {a.ctx}), {reps} repeats, "
+                         f"{sec * reps:.1f} s of CPU work; GB/s of the same byte model"}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC,
+        "value": round(gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": a.steps,
+        "warmup": max(3, a.warmup),
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if elem == 2 else "fp8_e4m3 KV, bf16 q/out, fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) q/k/v, shuffled page pool with 25% unused pages)",
+        "config": {
+            "workload": workload_name(a),
+            "B_per_gpu": B, "global_batch": B * world, "ctx": a.ctx, "Hq": Hq, "Hk": Hk,
+            "head_dim": D, "page_size": P, "num_splits": S, "pack_gqa": pack,
+            "parallelism": f"dp{world} (independent batches, no collective)",
+            "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step per GPU vs 126 MB L2; "
+                  "KV loads carry an L2 evict-first hint",
+            "algorithmic_bytes_per_step": step_bytes,
+        },
+        "pct_of_hbm_peak": round(100 * gbs / world / peak, 2),
+        "queries_per_s": round(world * B / (ms * 1e-3), 1),
+        "head_queries_per_s": round(world * B * Hq / (ms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(kern_gbs, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(kern_gbs / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "decode_kernel (call time minus the separately timed lse_combine)",
+                     "kernel_ms": round(kern_ms, 5), "combine_ms": round(comb_ms, 5)},
+        "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
+                "note": "q, page table and seq_lens H2D from pinned memory, out+lse D2H, "
+                        "KV cache device-resident"},
+        "gpu_launches": a.steps * (2 if S > 1 else 1),
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def reference_arm(a, world):
+    """The fp64 CPU oracle, timed on the host cores, on a bounded sample of the same
+    workload (rank 0 only)."""
+    import torch  # noqa: F401  (input generation)
+    from gqa_attention_paged_b200 import inputs
+
+    case = inputs.sweep_decode(a.B, seed=a.seed, ctx=a.ctx, kv_dtype=a.kv)
+    elem = 1 if a.kv == "fp8_e4m3" else 2
+    rows = [0, 1]
+    per_step = []
+    cores = 1
+    for _ in range(max(1, a.warmup) // 3):
+        run_oracle_sample(case, rows, 0.0)
+    for _ in range(a.steps):
+        sec, reps, cores = run_oracle_sample(case, rows, 0.0)
+        per_step.append(sec)
+    sec = sum(per_step) / len(per_step)
+    lens = [int(x) for x in case.kv.seq_lens]
+    sb = decode_step_bytes([lens[r] for r in rows], 32, 8, 128, elem, 16)
+    v = sb / sec / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(sec * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": workload_name(a), "B_per_gpu": a.B, "ctx": a.ctx,
+                   "sample": f"{len(rows)} of {a.B} sequences per step"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{len(rows)} of {a.B} sequences per step, {a.steps} steps"},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,264 @@
+"""Thin ctypes binding of libgqa_paged.so (include/gqa_paged.h).
+
+Argument marshalling only: torch tensors are checked for device, dtype, shape and
+contiguity and passed as raw device pointers with the current CUDA stream; every step of
+the computation runs in the library's kernels.  There is no fallback: if the library is
+missing or the tensors are not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from . import build as _build
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgqa_paged.so")
+
+GQA_OK = 0
+GQA_KV_BF16 = 0
+GQA_KV_FP8_E4M3 = 1
+GQA_MAX_SPLITS = 64
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+# name -> (restype, argtypes); the exported symbols of include/gqa_paged.h
+SIGNATURES = {
+    "gqa_paged_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "gqa_pick_splits": (_I, [_I, _I, _I, _I, _I]),
+    "gqa_paged_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                              ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
+    "gqa_paged_prefill_workspace_size": (_SZ, [_I, _I, _I]),
+    "gqa_paged_prefill": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                               ctypes.c_float, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
+    "gqa_paged_gather": (_I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "gqa_get_error": (_I, [_P, _P]),
+    "gqa_status_string": (ctypes.c_char_p, [_I]),
+}
+
+
+class GQAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+
+
+def load(path: Optional[str] = None):
+    """Load the library (building it first if the sources are newer).  Raises when it
+    cannot be built or loaded."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if path is None and (not os.path.exists(p) or _build._stale()):
+        _build.build()
+    if not os.path.exists(p):
+        raise RuntimeError(f"libgqa_paged.so not found at {p}: the CUDA extension is required")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().gqa_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != GQA_OK:
+        raise GQAError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+_KV_DTYPES = (torch.bfloat16, torch.uint8, torch.float8_e4m3fn)
+
+
+def _kv_code(t: torch.Tensor) -> int:
+    return GQA_KV_BF16 if t.dtype == torch.bfloat16 else GQA_KV_FP8_E4M3
+
+
+# ------------------------------------------------------------------------ raw ABI names
+
+def gqa_pick_splits(B: int, Hk: int, max_seq_len: int, page_size: int, kv_dtype: int = 0) -> int:
+    return load().gqa_pick_splits(B, Hk, max_seq_len, page_size, kv_dtype)
+
+
+def gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size, max_seq_len, kv_dtype,
+                                    num_splits) -> int:
+    return load().gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size, max_seq_len,
+                                                  kv_dtype, num_splits)
+
+
+def gqa_paged_prefill_workspace_size(total_q, Hq, head_dim) -> int:
+    return load().gqa_paged_prefill_workspace_size(total_q, Hq, head_dim)
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled, 256-byte aligned workspace of at least nbytes."""
+    n = (max(int(nbytes), 256) + 255) // 256 * 256
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gqa_paged_decode(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                     page_table: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                     num_splits: int = 0, pack_gqa: bool = True,
+                     k_scale: Optional[torch.Tensor] = None,
+                     v_scale: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, want_lse: bool = True,
+                     stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Paged GQA decode.  q bf16 [B][Hq][D]; pools [num_pages][Hk][P][D] bf16 or e4m3
+    (uint8/float8_e4m3fn with fp32 scales [num_pages][Hk]); page_table int32 [B][pt_stride];
+    seq_lens int32 [B].  Returns (out bf16 [B][Hq][D], lse fp32 [B][Hq] or None)."""
+    _need(q, "q", torch.bfloat16)
+    B, Hq, D = q.shape
+    _need(k_pages, "k_pages", _KV_DTYPES)
+    _need(v_pages, "v_pages", k_pages.dtype, k_pages.shape)
+    num_pages, Hk, P, D2 = k_pages.shape
+    if D2 != D:
+        raise ValueError("head_dim of q and the KV pools differ")
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B][pt_stride]")
+    kv_dtype = _kv_code(k_pages)
+    if kv_dtype == GQA_KV_FP8_E4M3:
+        if k_scale is None or v_scale is None:
+            raise ValueError("fp8 KV needs k_scale and v_scale")
+        _need(k_scale, "k_scale", torch.float32, (num_pages, Hk))
+        _need(v_scale, "v_scale", torch.float32, (num_pages, Hk))
+    pt_stride = page_table.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq))
+    need = gqa_paged_decode_workspace_size(B, Hq, Hk, D, P, pt_stride * P, kv_dtype, num_splits)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = load().gqa_paged_decode(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale), kv_dtype,
+        _ptr(page_table), pt_stride, _ptr(seq_lens), B, Hq, Hk, D, P, num_pages, float(scale),
+        int(num_splits), int(bool(pack_gqa)), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check("gqa_paged_decode", st)
+    return out, lse
+
+
+def gqa_paged_prefill(q: torch.Tensor, cu_q: torch.Tensor, k_pages: torch.Tensor,
+                      v_pages: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
+                      scale: float, max_q_len: int, causal: bool = True,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, want_lse: bool = True,
+                      stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Causal chunked prefill.  q bf16 [total_q][Hq][D]; cu_q int32 [B+1]; bf16 pools."""
+    _need(q, "q", torch.bfloat16)
+    T, Hq, D = q.shape
+    _need(k_pages, "k_pages", torch.bfloat16)
+    _need(v_pages, "v_pages", torch.bfloat16, k_pages.shape)
+    num_pages, Hk, P, D2 = k_pages.shape
+    if D2 != D:
+        raise ValueError("head_dim of q and the KV pools differ")
+    B = seq_lens.shape[0]
+    _need(cu_q, "cu_q", torch.int32, (B + 1,))
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    pt_stride = page_table.shape[1]
+    if out is None:
+        out = torch.empty(T, Hq, D, dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (T, Hq, D))
+    if lse is None and want_lse:
+        lse = torch.empty(T, Hq, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (T, Hq))
+    if workspace is None:
+        workspace = new_workspace(gqa_paged_prefill_workspace_size(T, Hq, D), q.device)
+    st = load().gqa_paged_prefill(
+        _ptr(q), _ptr(cu_q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), pt_stride,
+        _ptr(seq_lens), B, Hq, Hk, D, P, num_pages, float(scale), int(bool(causal)), T,
+        int(max_q_len), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream))
+    _check("gqa_paged_prefill", st)
+    return out, lse
+
+
+def lse_combine(o_part: torch.Tensor, lse_part: torch.Tensor,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Merge split results: o_part fp32 [S][rows][D], lse_part fp32 [S][rows]."""
+    _need(o_part, "o_part", torch.float32)
+    S, rows, D = o_part.shape
+    _need(lse_part, "lse_part", torch.float32, (S, rows))
+    if out is None:
+        out = torch.empty(rows, D, dtype=torch.bfloat16, device=o_part.device)
+    _need(out, "out", torch.bfloat16, (rows, D))
+    if lse is None:
+        lse = torch.empty(rows, dtype=torch.float32, device=o_part.device)
+    _need(lse, "lse", torch.float32, (rows,))
+    st = load().lse_combine(_ptr(o_part), _ptr(lse_part), S, rows, D, _ptr(out), _ptr(lse),
+                            _stream(stream))
+    _check("lse_combine", st)
+    return out, lse
+
+
+def gqa_paged_gather(k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+                     seq_lens: torch.Tensor, cu_kv: torch.Tensor, total: int,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Bit-exact copy-out of the paged cache: returns (k, v) [total][Hk][D]."""
+    _need(k_pages, "k_pages", _KV_DTYPES)
+    _need(v_pages, "v_pages", k_pages.dtype, k_pages.shape)
+    num_pages, Hk, P, D = k_pages.shape
+    B = seq_lens.shape[0]
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(cu_kv, "cu_kv", torch.int64, (B + 1,))
+    ko = torch.empty(total, Hk, D, dtype=k_pages.dtype, device=k_pages.device)
+    vo = torch.empty_like(ko)
+    st = load().gqa_paged_gather(_ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                                 page_table.shape[1], _ptr(seq_lens), _ptr(cu_kv), B, Hk, D, P,
+                                 num_pages, k_pages.element_size(), _ptr(ko), _ptr(vo),
+                                 _stream(stream))
+    _check("gqa_paged_gather", st)
+    return ko, vo
+
+
+def gqa_get_error(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream, return and clear the device error word of `workspace`."""
+    _need(workspace, "workspace", torch.uint8)
+    return load().gqa_get_error(_ptr(workspace), _stream(stream))

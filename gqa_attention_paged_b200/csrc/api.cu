@@ -1,0 +1,237 @@
+// api.cu -- the C ABI of libgqa_paged.so (declared in include/gqa_paged.h): argument
+// validation, workspace layout, TMA tensor-map encoding and kernel dispatch.  No device
+// memory is allocated here; every buffer is the caller's.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "gqa_internal.h"
+#include "gqa_paged.h"
+
+using namespace gqa;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool aligned(const void *p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// 2-D view [rows][D] of a KV pool, box = (128 bytes of a row) x 16 rows, 128B swizzle.
+int encode_kv_map(CUtensorMap *map, const void *pages, int kv_dtype, int D, int64_t rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return GQA_ERR_LAUNCH;
+    const int elt = kv_dtype == GQA_KV_FP8_E4M3 ? 1 : 2;
+    cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)D * elt};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / elt), (cuuint32_t)kDecodeTileTokens};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(map,
+                     elt == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(pages), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_LAUNCH;
+}
+
+bool valid_page_size(int P) { return P == 16 || P == 32 || P == 64; }
+
+int resolve_splits(int num_splits, int B, int Hk, int pt_stride, int P, int kv_dtype) {
+    if (num_splits > 0) return num_splits;
+    return gqa_pick_splits(B, Hk, pt_stride * P, P, kv_dtype);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gqa_status_string(int s) {
+    switch (s) {
+        case GQA_OK: return "ok";
+        case GQA_ERR_NULL: return "a required pointer is NULL";
+        case GQA_ERR_SHAPE: return "unsupported or inconsistent sizes";
+        case GQA_ERR_DTYPE: return "unsupported kv dtype / missing fp8 scales";
+        case GQA_ERR_SPLITS: return "num_splits out of range";
+        case GQA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case GQA_ERR_LAUNCH: return "CUDA launch or driver call failed";
+        case GQA_ERR_BAD_PAGE: return "page-table entry or sequence length out of range";
+        case GQA_ERR_TIMEOUT: return "a bounded device wait ran out";
+        case GQA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype) {
+    (void)kv_dtype;
+    if (B <= 0 || Hk <= 0 || page_size <= 0) return 1;
+    const int pages = (max_seq_len + page_size - 1) / page_size;
+    const int tiles = (max_seq_len + 15) / 16;
+    const int units = B * Hk;
+    const int slots = 148 * 3;  // SMs x resident decode CTAs per SM
+    // enough CTAs for ~4 waves, but keep >= 16 tiles of work per split
+    int s = (4 * slots + units - 1) / units;
+    const int max_by_work = tiles / 16 > 0 ? tiles / 16 : 1;
+    if (s > max_by_work) s = max_by_work;
+    if (s > pages) s = pages > 0 ? pages : 1;
+    if (s > GQA_MAX_SPLITS) s = GQA_MAX_SPLITS;
+    return s < 1 ? 1 : s;
+}
+
+size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int page_size,
+                                       int max_seq_len, int kv_dtype, int num_splits) {
+    int S = num_splits > 0 ? num_splits
+                           : gqa_pick_splits(B, Hk, max_seq_len, page_size, kv_dtype);
+    size_t bytes = kWorkspaceHeader;
+    if (S > 1) {
+        const size_t rows = (size_t)B * Hq;
+        bytes += align_up((size_t)S * rows * head_dim * sizeof(float), 256);
+        bytes += align_up((size_t)S * rows * sizeof(float), 256);
+    }
+    return bytes;
+}
+
+size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim) {
+    (void)total_q;
+    (void)Hq;
+    (void)head_dim;
+    return kWorkspaceHeader;
+}
+
+int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
+                     const float *k_scale, const float *v_scale, int kv_dtype,
+                     const int32_t *page_table, int pt_stride, const int32_t *seq_lens, int B,
+                     int Hq, int Hk, int head_dim, int page_size, int num_pages, float scale,
+                     int num_splits, int pack_gqa, void *out, float *lse, void *workspace,
+                     size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !workspace)
+        return GQA_ERR_NULL;
+    if (kv_dtype != GQA_KV_BF16 && kv_dtype != GQA_KV_FP8_E4M3) return GQA_ERR_DTYPE;
+    if (kv_dtype == GQA_KV_FP8_E4M3 && (!k_scale || !v_scale || head_dim != 128))
+        return GQA_ERR_DTYPE;
+    if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || Hk > 65535 ||
+        (head_dim != 64 && head_dim != 128) || !valid_page_size(page_size) || num_pages <= 0 ||
+        pt_stride <= 0 || (int64_t)num_pages * Hk * page_size > INT32_MAX ||
+        (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+        !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+        return GQA_ERR_ALIGN;
+    const int S = resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
+    const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                        pt_stride * page_size, kv_dtype, S);
+    if (!aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
+    if (B == 0) return GQA_OK;
+
+    const int64_t rows = (int64_t)num_pages * Hk * page_size;
+    CUtensorMap kmap, vmap;
+    if (encode_kv_map(&kmap, k_pages, kv_dtype, head_dim, rows) != GQA_OK ||
+        encode_kv_map(&vmap, v_pages, kv_dtype, head_dim, rows) != GQA_OK)
+        return GQA_ERR_LAUNCH;
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    DecodeArgs a;
+    a.q = q;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.page_table = page_table;
+    a.pt_stride = pt_stride;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hk = Hk;
+    a.D = head_dim;
+    a.P = page_size;
+    a.num_pages = num_pages;
+    a.kv_dtype = kv_dtype;
+    a.scale = scale;
+    a.num_splits = S;
+    a.pack_gqa = pack_gqa ? 1 : 0;
+    a.out = out;
+    a.lse = lse;
+    a.err = reinterpret_cast<int *>(ws);
+    const size_t rows_q = (size_t)B * Hq;
+    a.o_part = S > 1 ? reinterpret_cast<float *>(ws + kWorkspaceHeader) : nullptr;
+    a.lse_part = S > 1 ? reinterpret_cast<float *>(
+                             ws + kWorkspaceHeader +
+                             align_up((size_t)S * rows_q * head_dim * sizeof(float), 256))
+                       : nullptr;
+    if (launch_decode(a, kmap, vmap, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (S > 1 && launch_lse_combine(a.o_part, a.lse_part, S, (int)rows_q, head_dim, out, lse,
+                                    stream) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    return GQA_OK;
+}
+
+int lse_combine(const float *o_part, const float *lse_part, int num_splits, int rows,
+                int head_dim, void *out, float *lse, cudaStream_t stream) {
+    if (!o_part || !lse_part || !out) return GQA_ERR_NULL;
+    if (rows < 0 || (head_dim != 64 && head_dim != 128)) return GQA_ERR_SHAPE;
+    if (num_splits < 1 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (!aligned(o_part, 16) || !aligned(out, 16) || !aligned(lse_part, 4) ||
+        (lse && !aligned(lse, 4)))
+        return GQA_ERR_ALIGN;
+    return launch_lse_combine(o_part, lse_part, num_splits, rows, head_dim, out, lse, stream) ==
+                   cudaSuccess
+               ? GQA_OK
+               : GQA_ERR_LAUNCH;
+}
+
+int gqa_paged_gather(const void *k_pages, const void *v_pages, const int32_t *page_table,
+                     int pt_stride, const int32_t *seq_lens, const int64_t *cu_kv, int B,
+                     int Hk, int head_dim, int page_size, int num_pages, int elem_bytes,
+                     void *k_out, void *v_out, cudaStream_t stream) {
+    if (!k_pages || !v_pages || !page_table || !seq_lens || !cu_kv || !k_out || !v_out)
+        return GQA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hk <= 0 || (head_dim != 64 && head_dim != 128) ||
+        !valid_page_size(page_size) || num_pages <= 0 || pt_stride <= 0 ||
+        (elem_bytes != 1 && elem_bytes != 2))
+        return GQA_ERR_SHAPE;
+    if (!aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(k_out, 16) ||
+        !aligned(v_out, 16) || !aligned(cu_kv, 8))
+        return GQA_ERR_ALIGN;
+    if (B == 0) return GQA_OK;
+    return launch_gather(k_pages, v_pages, page_table, pt_stride, seq_lens, cu_kv, B, Hk,
+                         head_dim, page_size, num_pages, elem_bytes, k_out, v_out, stream) ==
+                   cudaSuccess
+               ? GQA_OK
+               : GQA_ERR_LAUNCH;
+}
+
+int gqa_get_error(void *workspace, cudaStream_t stream) {
+    if (!workspace) return GQA_ERR_NULL;
+    int err = 0;
+    if (cudaMemcpyAsync(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    if (err != 0) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(int), stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess)
+            return GQA_ERR_LAUNCH;
+    }
+    return err;
+}
+
+}  // extern "C"

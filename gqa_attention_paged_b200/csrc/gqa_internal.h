@@ -1,0 +1,66 @@
+// gqa_internal.h -- host-side interfaces between the C-ABI layer (api.cu) and the kernel
+// launchers (decode.cu, combine.cu, gather.cu, prefill.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gqa {
+
+constexpr size_t kWorkspaceHeader = 256;  // bytes before any scratch: holds the error word
+
+struct DecodeArgs {
+    const void *q;
+    const float *k_scale, *v_scale;
+    const int32_t *page_table;
+    int pt_stride;
+    const int32_t *seq_lens;
+    int B, Hq, Hk, D, P, num_pages;
+    int kv_dtype;
+    float scale;
+    int num_splits;
+    int pack_gqa;
+    void *out;
+    float *lse;
+    float *o_part, *lse_part;  // scratch for num_splits > 1
+    int *err;
+};
+
+// Launch the decode kernel (and nothing else) on `stream`.  The tensor maps describe the
+// K and V pools as 2-D arrays [num_pages*Hk*P rows][D].
+cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                          cudaStream_t stream);
+
+cudaError_t launch_lse_combine(const float *o_part, const float *lse_part, int num_splits,
+                               int rows, int D, void *out, float *lse, cudaStream_t stream);
+
+cudaError_t launch_gather(const void *k_pages, const void *v_pages, const int32_t *page_table,
+                          int pt_stride, const int32_t *seq_lens, const int64_t *cu_kv, int B,
+                          int Hk, int D, int P, int num_pages, int elem_bytes, void *k_out,
+                          void *v_out, cudaStream_t stream);
+
+struct PrefillArgs {
+    const void *q;
+    const int32_t *cu_q;
+    const int32_t *page_table;
+    int pt_stride;
+    const int32_t *seq_lens;
+    int B, Hq, Hk, D, P, num_pages;
+    float scale;
+    int causal;
+    int total_q, max_q_len;
+    void *out;
+    float *lse;
+    int *err;
+};
+
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap,
+                           const CUtensorMap &vmap, const CUtensorMap &qmap,
+                           cudaStream_t stream);
+
+// Box sizes the tensor maps must be encoded with.
+constexpr int kDecodeTileTokens = 16;
+
+}  // namespace gqa

@@ -1,0 +1,102 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports every function
+include/gqa_paged.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gqa_attention_paged_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                             src, flags=re.M):
+            names.append(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for n in ["gqa_paged_decode", "gqa_paged_prefill", "lse_combine", "gqa_paged_gather",
+              "gqa_get_error", "gqa_pick_splits", "gqa_paged_decode_workspace_size",
+              "gqa_paged_prefill_workspace_size", "gqa_status_string"]:
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol():
+    lib = binding.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"missing export {name}"
+        assert name in binding.SIGNATURES, f"binding lacks {name}"
+
+
+def test_library_has_no_oracle_or_torch_dependency():
+    """The product library links neither the oracle nor torch."""
+    lib_path = binding.LIB_PATH
+    binding.load()
+    data = open(lib_path, "rb").read()
+    assert b"oracle_decode" not in data and b"liboracle" not in data
+    assert b"libtorch" not in data and b"libc10" not in data
+
+
+def _fake(n=0x10000):
+    return ctypes.c_void_p(n)
+
+
+def _decode(**kw):
+    args = dict(q=_fake(), k=_fake(), v=_fake(), ks=None, vs=None, kvd=0, pt=_fake(), pts=8,
+                sl=_fake(), B=2, Hq=8, Hk=2, D=64, P=16, npg=16, scale=0.125, S=1, pack=1,
+                out=_fake(), lse=None, ws=_fake(), wsb=1 << 20, st=None)
+    args.update(kw)
+    return binding.load().gqa_paged_decode(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), -1), (dict(pt=None), -1), (dict(ws=None), -1),
+    (dict(Hq=6, Hk=4), -2), (dict(D=96), -2), (dict(P=8), -2), (dict(P=128), -2),
+    (dict(npg=0), -2), (dict(pts=0), -2), (dict(B=-1), -2), (dict(B=70000), -2),
+    (dict(kvd=5), -3), (dict(kvd=1), -3), (dict(kvd=1, ks=_fake(), vs=_fake(), D=64), -3),
+    (dict(S=-1), -4), (dict(S=65), -4),
+    (dict(q=_fake(0x10008)), -9), (dict(k=_fake(0x10004)), -9),
+    (dict(ws=_fake(0x10010)), -5), (dict(wsb=16), -5),
+    (dict(S=4, wsb=256), -5),
+])
+def test_decode_rejects_bad_arguments_on_the_host(kw, status):
+    assert _decode(**kw) == status
+
+
+def test_host_helpers():
+    lib = binding.load()
+    assert lib.gqa_paged_decode_workspace_size(4, 8, 2, 64, 16, 256, 0, 1) == 256
+    assert lib.gqa_paged_decode_workspace_size(4, 8, 2, 64, 16, 256, 0, 3) == \
+        256 + 3 * 32 * 64 * 4 + 512
+    for B in (1, 16, 64, 256):
+        s = lib.gqa_pick_splits(B, 8, 2048, 16, 0)
+        assert 1 <= s <= 64
+    assert lib.gqa_pick_splits(1, 8, 16, 16, 0) == 1
+    assert binding.status_string(-7).startswith("page-table")
+    assert lib.lse_combine(None, _fake(), 2, 4, 64, _fake(), None, None) == -1
+    assert lib.lse_combine(_fake(), _fake(), 0, 4, 64, _fake(), None, None) == -4
+    assert lib.lse_combine(_fake(), _fake(), 2, 4, 32, _fake(), None, None) == -2
+    assert lib.gqa_paged_gather(_fake(), _fake(), _fake(), 4, _fake(), _fake(), 2, 2, 64, 16, 8,
+                                3, _fake(), _fake(), None) == -2
+    assert lib.gqa_get_error(None, None) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    kp = torch.zeros(4, 2, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.gqa_paged_decode(q, kp, kp, torch.zeros(1, 4, dtype=torch.int32),
+                                 torch.ones(1, dtype=torch.int32), 0.125)

@@ -351,3 +351,17 @@ def test_kv_bytes_model_matches_the_pages_figure():
     mha = bench.decode_kv_bytes([2048] * 4, Hk=fx["Hq"], D=128, elem=2)
     assert gqa / mha == fx["kv_bytes_ratio_gqa_over_mha"]
     assert 1 - gqa / mha == fx["kv_reduction"]
+
+
+def test_fp8_quantisation_error_sets_the_fp8_bound():
+    """On the 70B-shaped long-context workload (1% outliers at 8 sigma), exact fp64
+    attention over the dequantised e4m3 cache differs from attention over the unquantised
+    values by ~2e-2: below the 5e-2 max-|err| bound adopted for the fp8 path, and above
+    2e-3 + 5e-2|ref| in some elements, so that per-element form cannot be met by any
+    implementation and is not the gate."""
+    case = inputs.long70b_decode(seed=0, kv_dtype="fp8_e4m3")
+    deq, _ = oracle_decode(case)
+    ref, _ = oracle_decode(case, use_bf16_pool=True)
+    d = np.abs(deq - ref)
+    assert 5e-3 < d.max() <= 5e-2
+    assert (d > 2e-3 + 5e-2 * np.abs(ref)).any()
