@@ -55,6 +55,20 @@ int encode_kv_map(CUtensorMap *map, const void *pages, int kv_dtype, int D, int6
     return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_LAUNCH;
 }
 
+// 3-D view [total_q][Hq][D] of q (or out), box = 64 dims x g heads x T tokens, 128B swizzle.
+int encode_q_map(CUtensorMap *map, const void *q, int total_q, int Hq, int D, int g, int T) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return GQA_ERR_LAUNCH;
+    cuuint64_t gdim[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)total_q};
+    cuuint64_t gstride[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)T};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), gdim, gstride,
+                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_LAUNCH;
+}
+
 bool valid_page_size(int P) { return P == 16 || P == 32 || P == 64; }
 
 int resolve_splits(int num_splits, int B, int Hk, int pt_stride, int P, int kv_dtype) {
@@ -182,6 +196,58 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                                     stream) != cudaSuccess)
         return GQA_ERR_LAUNCH;
     return GQA_OK;
+}
+
+int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
+                      const void *v_pages, const int32_t *page_table, int pt_stride,
+                      const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim,
+                      int page_size, int num_pages, float scale, int causal, int total_q,
+                      int max_q_len, void *out, float *lse, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !cu_q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !workspace)
+        return GQA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || Hk > 65535 ||
+        Hq / Hk > 128 || head_dim != 128 || !valid_page_size(page_size) || num_pages <= 0 ||
+        pt_stride <= 0 || total_q < 0 || max_q_len < 0 ||
+        (int64_t)num_pages * Hk * page_size > INT32_MAX ||
+        (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+        !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(cu_q, 4) ||
+        (lse && !aligned(lse, 4)))
+        return GQA_ERR_ALIGN;
+    if (!aligned(workspace, 256) ||
+        workspace_bytes < gqa_paged_prefill_workspace_size(total_q, Hq, head_dim))
+        return GQA_ERR_WORKSPACE;
+    if (B == 0 || total_q == 0 || max_q_len == 0) return GQA_OK;
+    const int g = Hq / Hk;
+    const int T = 128 / g;
+    const int64_t rows = (int64_t)num_pages * Hk * page_size;
+    CUtensorMap kmap, vmap, qmap;
+    if (encode_kv_map(&kmap, k_pages, GQA_KV_BF16, head_dim, rows) != GQA_OK ||
+        encode_kv_map(&vmap, v_pages, GQA_KV_BF16, head_dim, rows) != GQA_OK ||
+        encode_q_map(&qmap, q, total_q, Hq, head_dim, g, T) != GQA_OK)
+        return GQA_ERR_LAUNCH;
+    PrefillArgs a;
+    a.q = q;
+    a.cu_q = cu_q;
+    a.page_table = page_table;
+    a.pt_stride = pt_stride;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hk = Hk;
+    a.D = head_dim;
+    a.P = page_size;
+    a.num_pages = num_pages;
+    a.scale = scale;
+    a.causal = causal ? 1 : 0;
+    a.total_q = total_q;
+    a.max_q_len = max_q_len;
+    a.out = out;
+    a.lse = lse;
+    a.err = reinterpret_cast<int *>(workspace);
+    return launch_prefill(a, kmap, vmap, qmap, stream) == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
 }
 
 int lse_combine(const float *o_part, const float *lse_part, int num_splits, int rows,

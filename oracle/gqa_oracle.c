@@ -250,7 +250,9 @@ void oracle_decode_split(const uint16_t *q, const void *k_pages, const void *v_p
 }
 
 /* Merge of split results by log-sum-exp: M = max_s lse_s, w_s = exp(lse_s - M),
- * O = sum w_s o_s / sum w_s, lse = M + ln sum w_s.  All splits empty: O = 0, lse = -inf.
+ * O = sum w_s o_s / sum w_s, lse = M + ln sum w_s, the sums running over the non-empty
+ * splits only: an empty split (lse = -inf) has no tokens, hence no output to weigh (its
+ * o_s is undefined), and is left out.  All splits empty: O = 0, lse = -inf.
  * o_part [S][rows][D], lse_part [S][rows]. */
 void oracle_lse_combine(const double *o_part, const double *lse_part, int S, int rows, int D,
                         double *out, double *lse)
@@ -268,6 +270,8 @@ void oracle_lse_combine(const double *o_part, const double *lse_part, int S, int
         }
         double W = 0.0;
         for (int s = 0; s < S; ++s) {
+            if (lse_part[(int64_t)s * rows + r] == -INFINITY)
+                continue;
             double w = exp(lse_part[(int64_t)s * rows + r] - M);
             W += w;
             for (int d = 0; d < D; ++d)

@@ -34,6 +34,7 @@ MUTANTS = {
     "query_head_index": ("qd[d] = oracle_bf16_to_f64(q[((int64_t)b * Hq + h) * D + d]);",
                          "qd[d] = oracle_bf16_to_f64(q[((int64_t)b * Hq + j) * D + d]);"),
     "fp8_scale_ignored": ("* scale[phys * Hk + kvh];", ";"),
+    "empty_split_weighed": ("if (lse_part[(int64_t)s * rows + r] == -INFINITY)\n                continue;", ""),
 }
 
 

@@ -203,6 +203,22 @@ def test_lse_combine_all_empty_rows():
     assert lse[2] == 0.5
 
 
+def test_lse_combine_leaves_out_empty_splits():
+    """An empty split (lse = -inf) carries no tokens: whatever its partial holds (even
+    NaN), the merge equals the merge of the other splits."""
+    rng = np.random.default_rng(1)
+    o = rng.normal(size=(3, 4, 8))
+    l = rng.normal(size=(3, 4))
+    ref, ref_l = oracle.lse_combine(o[[0, 2]], l[[0, 2]])
+    o2 = o.copy()
+    l2 = l.copy()
+    l2[1] = -np.inf
+    o2[1] = np.nan
+    out, lse = oracle.lse_combine(o2, l2)
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(lse, ref_l)
+
+
 def test_physical_page_permutation_invariance():
     case = inputs.make_decode_case(3, 8, 2, 64, 16, [40, 77, 128], seed=9)
     out, lse = oracle_decode(case)
