@@ -45,6 +45,27 @@ def decode_step_bytes(seq_lens, Hq, Hk, D, elem, P=16):
     return b
 
 
+def rank_seed(seed, rank):
+    """Each rank of a weak-scaling run draws its own batch."""
+    return seed + rank
+
+
+def max_over_ranks(x, dist=None, device="cpu"):
+    """Max of a per-rank scalar over all ranks (every rank gets it)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(step_bytes_per_rank, world, ms_max):
+    """Whole-job GB/s: every rank moves step_bytes_per_rank per step; the job's step time
+    is the slowest rank's."""
+    return world * step_bytes_per_rank / (ms_max * 1e-3) / 1e9
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -215,7 +236,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    case = inputs.sweep_decode(a.B, seed=a.seed + rank, ctx=a.ctx, kv_dtype=a.kv)
+    case = inputs.sweep_decode(a.B, seed=rank_seed(a.seed, rank), ctx=a.ctx, kv_dtype=a.kv)
     kv = case.kv
     q = case.q.to(dev)
     kp, vp = kv.k_pages.to(dev), kv.v_pages.to(dev)
@@ -243,13 +264,6 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # parity spot check of this exact launch configuration before timing
     step()
     torch.cuda.synchronize(dev)
@@ -270,7 +284,7 @@ def main():
     barrier()
     ms = ev0.elapsed_time(ev1) / a.steps
     clk = clocks.stop()
-    ms = max_over_ranks(ms)
+    ms = max_over_ranks(ms, dist, dev)
 
     # The dominant kernel alone: time the merge kernel by itself on the same partials and
     # subtract it (when the call splits), all with events on this stream.
@@ -323,14 +337,14 @@ def main():
         e2e_step()
     e1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / a.steps)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dist, dev)
 
     lens = [int(x) for x in kv.seq_lens]
     step_bytes = decode_step_bytes(lens, Hq, Hk, D, elem, P)
     peak, peak_kind = peaks()
-    gbs = world * step_bytes / (ms * 1e-3) / 1e9
+    gbs = aggregate_gbs(step_bytes, world, ms)
     kern_gbs = step_bytes / (kern_ms * 1e-3) / 1e9
-    e2e_gbs = world * step_bytes / (e2e_ms * 1e-3) / 1e9
+    e2e_gbs = aggregate_gbs(step_bytes, world, e2e_ms)
     wkey = f"B{B}_ctx{a.ctx}_{a.kv}_S{S}_pack{int(pack)}"
     traffic = traffic_from_profile(wkey)
 

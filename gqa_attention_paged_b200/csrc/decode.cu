@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 3)
         // ---- online softmax (exp2 domain), per packed head column
         const float kmul = FP8 ? scale_log2 * sm.kscale[stage] / qmul : scale_log2;
         const bool v0 = gq < valid, v1 = gq + 8 < valid;
-        uint32_t pb[NT][2];
+        uint32_t pb[NT][2], pbl[NT][2];
         float alpha[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -334,8 +334,15 @@ __global__ void __launch_bounds__(kThreads, 3)
                 m[nt][jj] = mnew;
             }
             if (!FP8) {
-                pb[nt][0] = movmatrix_trans(pack_bf16(p[0], p[1]));
-                pb[nt][1] = movmatrix_trans(pack_bf16(p[2], p[3]));
+                // P as a bf16 value plus its bf16 residual: O += V^T P_hi^T + V^T P_lo^T keeps
+                // the weights at ~16 bits (one bf16 P would cost up to 2^-9 per weight).
+                uint32_t h0, l0, h1, l1;
+                split_bf16x2(p[0], p[1], h0, l0);
+                split_bf16x2(p[2], p[3], h1, l1);
+                pb[nt][0] = movmatrix_trans(h0);
+                pb[nt][1] = movmatrix_trans(h1);
+                pbl[nt][0] = movmatrix_trans(l0);
+                pbl[nt][1] = movmatrix_trans(l1);
             } else {
                 pb[nt][0] = movmatrix_trans(pack_f16(p[0], p[1]));
                 pb[nt][1] = movmatrix_trans(pack_f16(p[2], p[3]));
@@ -358,7 +365,10 @@ __global__ void __launch_bounds__(kThreads, 3)
                 uint32_t af[4];
                 ldsm_x4_trans(af, vbase + swz(r, (dt * 16 + (j & 1) * 8) * 2));
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16(o[nt][dt], af, pb[nt][0], pb[nt][1]);
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16(o[nt][dt], af, pb[nt][0], pb[nt][1]);
+                    mma_bf16(o[nt][dt], af, pbl[nt][0], pbl[nt][1]);
+                }
             }
         } else {
             // fp8 V: plain ldmatrix gives each lane 4 consecutive dims of one token;
@@ -411,8 +421,9 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (sm.abort_flag) return;
 
     constexpr int HW = 8 * NT;  // packed head columns per CTA
-    float *red_o = reinterpret_cast<float *>(&sm.tiles[0][0][0]);  // [warp][HW][D]
-    float *red_m = red_o + kConsumerWarps * HW * D;                 // [warp][HW]
+    constexpr int RS = D + 4;   // padded row: the 4 lanes sharing a dim hit 4 banks
+    float *red_o = reinterpret_cast<float *>(&sm.tiles[0][0][0]);  // [warp][HW][RS]
+    float *red_m = red_o + kConsumerWarps * HW * RS;                // [warp][HW]
     float *red_l = red_m + kConsumerWarps * HW;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -427,11 +438,11 @@ __global__ void __launch_bounds__(kThreads, 3)
                 d0 = dt * 16 + 4 * (gq >> 1) + (gq & 1);
                 d1 = d0 + 2;
             }
-            float *w = red_o + (size_t)(warp * HW + h0) * D;
+            float *w = red_o + (size_t)(warp * HW + h0) * RS;
             w[d0] = o[nt][dt][0];
-            w[D + d0] = o[nt][dt][1];
+            w[RS + d0] = o[nt][dt][1];
             w[d1] = o[nt][dt][2];
-            w[D + d1] = o[nt][dt][3];
+            w[RS + d1] = o[nt][dt][3];
         }
         if (gq == 0) {
             red_m[warp * HW + h0] = m[nt][0];
@@ -454,8 +465,8 @@ __global__ void __launch_bounds__(kThreads, 3)
             for (int w = 0; w < kConsumerWarps; ++w) {
                 const float f = fast_exp2(red_m[w * HW + h] - M);
                 Ls += f * red_l[w * HW + h];
-                o0 += f * red_o[(size_t)(w * HW + h) * D + d];
-                o1 += f * red_o[(size_t)(w * HW + h) * D + d + 1];
+                o0 += f * red_o[(size_t)(w * HW + h) * RS + d];
+                o1 += f * red_o[(size_t)(w * HW + h) * RS + d + 1];
             }
         }
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
@@ -477,7 +488,7 @@ template <int D, int NT, bool FP8>
 cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
     const size_t smem = sizeof(Smem<D, FP8>) + 1024;
-    static_assert(sizeof(float) * kConsumerWarps * 8 * NT * (D + 2) <=
+    static_assert(sizeof(float) * kConsumerWarps * 8 * NT * (D + 6) <=
                       sizeof(uint8_t) * Cfg<D, FP8>::kStages * 2 * Cfg<D, FP8>::kTileBytes,
                   "reduction area must fit in the stage ring");
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8>,

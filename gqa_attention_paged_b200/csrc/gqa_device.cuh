@@ -167,6 +167,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Two-term bf16 split of (lo, hi): hi_part + lo_part equals the fp32 inputs to ~16
+// significant bits, so a product with a bf16 operand keeps fp32-level accuracy.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat16 ah = __float2bfloat16_rn(a), bh = __float2bfloat16_rn(b);
+    __nv_bfloat162 h;
+    h.x = ah;
+    h.y = bh;
+    hi = *reinterpret_cast<uint32_t *>(&h);
+    lo = pack_bf16(a - __bfloat162float(ah), b - __bfloat162float(bh));
+}
+
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);

@@ -19,6 +19,9 @@
 //   warp 1   allocates tensor memory (S: 128 columns, O: 128 columns) and issues the MMAs
 //            (one thread), S_{j+1} overlapping the softmax of tile j.
 //   warps 2-5 softmax / correction / epilogue: thread = one row (tensor-memory lane).
+// P is written as a bf16 value plus its bf16 residual and O += P_hi V + P_lo V, so the
+// probabilities keep ~16 significant bits (a single bf16 P loses up to 2^-9 of each
+// weight, visible as ~5e-3 errors in short rows whose terms cancel).
 // The running max is only moved when a row's max grows by more than 2^8, so O (kept in
 // tensor memory) is rescaled rarely; the final O / l is exact for any reference max.
 // Every wait is bounded; on expiry the kernel records GQA_ERR_TIMEOUT, finishes its
@@ -47,7 +50,8 @@ struct alignas(1024) PSmem {
     uint8_t q[kTileBytesP];
     uint8_t k[kStages][kTileBytesP];
     uint8_t v[kStages][kTileBytesP];
-    uint8_t p[kTileBytesP];
+    uint8_t p[kTileBytesP];     // bf16 part of P
+    uint8_t p_lo[kTileBytesP];  // bf16 residual of P (P - p): two MMAs keep P at ~16 bits
     uint64_t q_full;
     uint64_t kv_full[kStages];
     uint64_t kv_empty[kStages];
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);   // Q, K both K-major
         constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, kD, 0, 1);   // P K-major, V MN-major
-        const uint32_t qa = smem_u32(sm.q), pa = smem_u32(sm.p);
+        const uint32_t qa = smem_u32(sm.q), pa = smem_u32(sm.p), pla = smem_u32(sm.p_lo);
         bool ok = wait_all(&sm.q_full, 0) && wait_all(&sm.kv_full[0], 0);
         int committed_pv = 0;  // PV MMAs committed to pv_done
         if (ok) {
@@ -239,6 +243,12 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     tc_mma_ss(tO, smem_desc_sw128(pa + aoff, 16, 1024),
                               smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                    tc_mma_ss(tO, smem_desc_sw128(pla + aoff, 16, 1024),
+                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
                 }
                 tc_commit(&sm.pv_done);
                 tc_commit(&sm.kv_empty[stage]);
@@ -314,9 +324,11 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     tmem_wait_st();
                 }
             }
-            // P row (bf16) into the swizzled K-major tile: 16 chunks of 8 keys.
+            // P row (bf16 value + bf16 residual) into the swizzled K-major tiles: 16 chunks
+            // of 8 keys each.
             float sum = 0.f;
             uint8_t *prow = sm.p + row * 128;
+            uint8_t *plrow = sm.p_lo + row * 128;
 #pragma unroll
             for (int ch = 0; ch < 16; ++ch) {
                 float pv[8];
@@ -325,13 +337,14 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     pv[e] = fast_exp2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + e]) - mref0);
                     sum += pv[e];
                 }
-                uint4 w;
-                w.x = pack_bf16(pv[0], pv[1]);
-                w.y = pack_bf16(pv[2], pv[3]);
-                w.z = pack_bf16(pv[4], pv[5]);
-                w.w = pack_bf16(pv[6], pv[7]);
-                *reinterpret_cast<uint4 *>(prow + (ch >> 3) * kHalfBytes +
-                                           (((ch & 7) ^ (row & 7)) << 4)) = w;
+                uint4 w, wl;
+                split_bf16x2(pv[0], pv[1], w.x, wl.x);
+                split_bf16x2(pv[2], pv[3], w.y, wl.y);
+                split_bf16x2(pv[4], pv[5], w.z, wl.z);
+                split_bf16x2(pv[6], pv[7], w.w, wl.w);
+                const int off = (ch >> 3) * kHalfBytes + (((ch & 7) ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4 *>(prow + off) = w;
+                *reinterpret_cast<uint4 *>(plrow + off) = wl;
             }
             l = l * alpha + sum;
             m_ref = new_ref;
