@@ -34,6 +34,8 @@ SIGNATURES = {
     "gqa_pick_splits": (_I, [_I, _I, _I, _I, _I]),
     "gqa_paged_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                               ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
+    "gqa_paged_decode_static_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
+                                             _I, _I, _I, ctypes.c_float, _I, _I, _P, _P, _P]),
     "gqa_paged_prefill_workspace_size": (_SZ, [_I, _I, _I]),
     "gqa_paged_prefill": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                ctypes.c_float, _I, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -178,6 +180,41 @@ def gqa_paged_decode(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tens
         int(num_splits), int(bool(pack_gqa)), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel(), _stream(stream))
     _check("gqa_paged_decode", st)
+    return out, lse
+
+
+def gqa_paged_decode_static_scratch(q: torch.Tensor, k_pages: torch.Tensor,
+                                    v_pages: torch.Tensor, page_table: torch.Tensor,
+                                    seq_lens: torch.Tensor, scale: float, num_splits: int = 0,
+                                    pack_gqa: bool = True,
+                                    k_scale: Optional[torch.Tensor] = None,
+                                    v_scale: Optional[torch.Tensor] = None,
+                                    out: Optional[torch.Tensor] = None,
+                                    lse: Optional[torch.Tensor] = None,
+                                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """gqa_paged_decode without a workspace: the library's fixed scratch array is used
+    (for callers that cannot allocate device memory; see include/gqa_paged.h).  `out` and
+    `lse` must be passed in by such callers; they are only created here for convenience."""
+    _need(q, "q", torch.bfloat16)
+    B, Hq, D = q.shape
+    _need(k_pages, "k_pages", _KV_DTYPES)
+    _need(v_pages, "v_pages", k_pages.dtype, k_pages.shape)
+    num_pages, Hk, P, _ = k_pages.shape
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    kv_dtype = _kv_code(k_pages)
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    st = load().gqa_paged_decode_static_scratch(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale), kv_dtype,
+        _ptr(page_table), page_table.shape[1], _ptr(seq_lens), B, Hq, Hk, D, P, num_pages,
+        float(scale), int(num_splits), int(bool(pack_gqa)), _ptr(out), _ptr(lse),
+        _stream(stream))
+    _check("gqa_paged_decode_static_scratch", st)
     return out, lse
 
 

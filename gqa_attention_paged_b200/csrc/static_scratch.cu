@@ -1,0 +1,68 @@
+// static_scratch.cu -- paged GQA decode for callers that cannot allocate device memory.
+//
+// gqa_paged_decode() takes its scratch (error word, split partials) from a workspace the
+// caller allocates.  gqa_paged_decode_static_scratch() runs the same decode with that
+// scratch in a fixed array compiled into this library instead, so the caller passes only
+// its inputs and outputs.  The array's device address is looked up once per device with
+// cudaGetSymbolAddress (the array's name is only a host-side stand-in in host code), and
+// the call then goes through gqa_paged_decode() unchanged.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "gqa_paged.h"
+
+namespace {
+
+// Scratch shared by every call of gqa_paged_decode_static_scratch on a device.  Every
+// GPU that loads this library holds these bytes until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[GQA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_lock;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up on first use).
+int scratch_address(void **addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_LAUNCH;
+    std::lock_guard<std::mutex> guard(g_lock);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+            return GQA_ERR_LAUNCH;
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" int gqa_paged_decode_static_scratch(
+    const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
+    const float *v_scale, int kv_dtype, const int32_t *page_table, int pt_stride,
+    const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim, int page_size, int num_pages,
+    float scale, int num_splits, int pack_gqa, void *out, float *lse, cudaStream_t stream) {
+    // Size check first (only for arguments gqa_paged_decode would accept; it reports the
+    // rest itself): the scratch this call needs must fit the fixed array.
+    if (B > 0 && Hq > 0 && Hk > 0 && head_dim > 0 && page_size > 0 && pt_stride > 0 &&
+        num_splits >= 0 && num_splits <= GQA_MAX_SPLITS &&
+        (int64_t)pt_stride * page_size <= INT32_MAX) {
+        const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                            pt_stride * page_size, kv_dtype,
+                                                            num_splits);
+        if (need > (size_t)GQA_STATIC_SCRATCH_BYTES) return GQA_ERR_WORKSPACE;
+    }
+    void *ws = nullptr;
+    const int st = scratch_address(&ws);
+    if (st != GQA_OK) return st;
+    // The array keeps the previous call's contents; only the error word must start at
+    // zero (the split partials are fully rewritten by every call that uses them).
+    if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return GQA_ERR_LAUNCH;
+    return gqa_paged_decode(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table,
+                            pt_stride, seq_lens, B, Hq, Hk, head_dim, page_size, num_pages, scale,
+                            num_splits, pack_gqa, out, lse, ws, (size_t)GQA_STATIC_SCRATCH_BYTES,
+                            stream);
+}

@@ -124,6 +124,51 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                      size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Largest scratch gqa_paged_decode_static_scratch() can use: its fixed array's size.
+ */
+#define GQA_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * gqa_paged_decode() without a workspace argument.  The pages have no counterpart: this is
+ * an interface convenience, and the computation is exactly gqa_paged_decode()'s.
+ *
+ * Who it is for: callers that cannot allocate device memory where they run decode.
+ * Examples are an inference-engine plugin whose enqueue step may not allocate, a loop
+ * with a real-time budget that forbids allocation after start-up, and a host whose
+ * device memory is all handed out by another allocator.  Such callers cannot create and
+ * own the workspace that gqa_paged_decode() needs for its split partials.
+ *
+ * How: the scratch (error word, then o_part / lse_part) lives in one fixed
+ * GQA_STATIC_SCRATCH_BYTES array compiled into this library (a `static __device__`
+ * array).  Every GPU that loads the library holds the array until the process exits.
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine is called.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it.  Make that first
+ *     call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the last call's contents.
+ *     Each call clears the error word (an async memset on `stream`) and fully rewrites
+ *     the partials it uses.  Calls that overlap on the GPU (other streams, other threads)
+ *     race on the array: serialise them.
+ *   - Device-side errors (out-of-range page entries, a bounded wait that ran out) are
+ *     recorded in the array's error word but cannot be read back through this entry
+ *     point.  Use gqa_paged_decode() with a workspace when those reports are needed.
+ *
+ * Arguments are gqa_paged_decode()'s, minus workspace / workspace_bytes.  Returns what
+ * gqa_paged_decode() returns.  Also returns GQA_ERR_WORKSPACE, with nothing enqueued,
+ * when the call needs more than GQA_STATIC_SCRATCH_BYTES of scratch, i.e. when
+ * gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+ * pt_stride * page_size, kv_dtype, num_splits) exceeds it.  Lower num_splits or the
+ * batch to fit.
+ */
+int gqa_paged_decode_static_scratch(const void *q, const void *k_pages, const void *v_pages,
+                                    const float *k_scale, const float *v_scale, int kv_dtype,
+                                    const int32_t *page_table, int pt_stride,
+                                    const int32_t *seq_lens, int B, int Hq, int Hk,
+                                    int head_dim, int page_size, int num_pages, float scale,
+                                    int num_splits, int pack_gqa, void *out, float *lse,
+                                    cudaStream_t stream);
+
+/*
  * Bytes of workspace gqa_paged_prefill() needs (the 256-byte error-word header).
  */
 size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim);
