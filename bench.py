@@ -246,7 +246,9 @@ def main():
     elem = 1 if a.kv == "fp8_e4m3" else 2
     B, Hq, Hk, D, P = a.B, 32, 8, 128, 16
     kvc = binding.GQA_KV_FP8_E4M3 if elem == 1 else binding.GQA_KV_BF16
-    S = a.splits if a.splits > 0 else binding.gqa_pick_splits(B, Hk, pt.shape[1] * P, P, kvc)
+    balanced = a.splits == 0 and B <= 2048  # num_splits = 0: the balanced persistent schedule
+    S = a.splits if a.splits > 0 else (0 if balanced else
+                                      binding.gqa_pick_splits(B, Hk, pt.shape[1] * P, P, kvc))
     pack = not a.no_pack
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
@@ -379,6 +381,7 @@ def main():
             "workload": workload_name(a),
             "B_per_gpu": B, "global_batch": B * world, "ctx": a.ctx, "Hq": Hq, "Hk": Hk,
             "head_dim": D, "page_size": P, "num_splits": S, "pack_gqa": pack,
+            "schedule": "balanced persistent (one launch)" if S == 0 else f"{S} splits + merge",
             "parallelism": f"dp{world} (independent batches, no collective)",
             "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step per GPU vs 126 MB L2; "
                   "KV loads carry an L2 evict-first hint",
@@ -391,7 +394,8 @@ def main():
                      "unit": "GB/s", "frac": round(kern_gbs / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "decode_kernel (call time minus the separately timed lse_combine)",
+                     "kernel": ("decode_sk_kernel (the whole call: one launch)" if S == 0 else
+                                "decode_kernel (call time minus the separately timed lse_combine)"),
                      "kernel_ms": round(kern_ms, 5), "combine_ms": round(comb_ms, 5)},
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),

@@ -76,6 +76,30 @@ int resolve_splits(int num_splits, int B, int Hk, int pt_stride, int P, int kv_d
     return gqa_pick_splits(B, Hk, pt_stride * P, P, kv_dtype);
 }
 
+bool use_stream_k(int num_splits, int B) { return num_splits == 0 && B <= kStreamMaxBatch; }
+
+// Merge-piece slots of the balanced schedule: 2 per worker, for the largest grid.
+size_t stream_k_piece_bytes(int Hq, int Hk, int D) {
+    const int g = Hq / Hk;
+    const int hpc = g < 16 ? g : 16;
+    const size_t slots = (size_t)kStreamMaxSms * kStreamCtasPerSm * kStreamWorkersPerCta * 2;
+    const size_t slot_floats = ((size_t)hpc * (D + 1) + 3) / 4 * 4;  // 16-byte aligned slots
+    return align_up(slots * slot_floats * sizeof(float), 256);
+}
+
+int sm_count() {
+    static int cached[256] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -114,6 +138,8 @@ int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype)
 
 size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int page_size,
                                        int max_seq_len, int kv_dtype, int num_splits) {
+    if (use_stream_k(num_splits, B) && Hq > 0 && Hk > 0 && Hq % Hk == 0)
+        return decode_zero_prefix_bytes(B, Hq) + stream_k_piece_bytes(Hq, Hk, head_dim);
     int S = num_splits > 0 ? num_splits
                            : gqa_pick_splits(B, Hk, max_seq_len, page_size, kv_dtype);
     size_t bytes = kWorkspaceHeader;
@@ -152,9 +178,11 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
     if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
         !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
         return GQA_ERR_ALIGN;
-    const int S = resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
+    const bool sk = use_stream_k(num_splits, B);
+    const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
     const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
-                                                        pt_stride * page_size, kv_dtype, S);
+                                                        pt_stride * page_size, kv_dtype,
+                                                        sk ? 0 : S);
     if (!aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
     if (B == 0) return GQA_OK;
 
@@ -191,6 +219,14 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                              ws + kWorkspaceHeader +
                              align_up((size_t)S * rows_q * head_dim * sizeof(float), 256))
                        : nullptr;
+    a.stream_k = sk ? 1 : 0;
+    a.counters = sk ? reinterpret_cast<int *>(ws + kWorkspaceHeader) : nullptr;
+    a.pieces = sk ? reinterpret_cast<float *>(ws + decode_zero_prefix_bytes(B, Hq)) : nullptr;
+    {
+        int sms = sm_count();
+        if (sms > kStreamMaxSms) sms = kStreamMaxSms;
+        a.grid = sms * kStreamCtasPerSm;
+    }
     if (launch_decode(a, kmap, vmap, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
     if (S > 1 && launch_lse_combine(a.o_part, a.lse_part, S, (int)rows_q, head_dim, out, lse,
                                     stream) != cudaSuccess)

@@ -1,19 +1,27 @@
-// decode.cu -- paged GQA decode kernel for sm_100a (bf16 and fp8-e4m3 KV).
+// decode.cu -- paged GQA decode kernels for sm_100a (bf16 and fp8-e4m3 KV).
 //
-// One CTA = (split, kv head [, head chunk], sequence).  It streams the split's KV tiles
-// (16 tokens of one page each) from the pool into a shared-memory ring with TMA tile
-// loads (128-byte swizzled, no multicast), and computes attention for ALL query heads
-// of the group at once (PackGQA: "解锁GQA性能潜力：从批量大小敏感性到高效优化实践",
-// section "核心参数调优：PackGQA与NumSplits的协同舞蹈"), so every KV byte crosses HBM
-// once.  Scores and P·V run on warp-level tensor cores (m16n8k16, fp32 accumulate) with
-// the tokens of a tile as the M dimension and the packed heads as N; the softmax is the
-// online (running max / running sum) form in fp32, exp2 domain, as in the tiled fused
-// attention of "TensorRT-LLM与TensorRT核心差异解析", section 4.2.1 FlashAttention.
+// Both kernels stream 16-token K/V tiles of one page and one kv head from the pool into a
+// shared-memory ring with TMA tile loads (128-byte swizzled, no multicast), and compute
+// attention for ALL query heads of the group per tile (PackGQA:
+// "解锁GQA性能潜力：从批量大小敏感性到高效优化实践", section
+// "核心参数调优：PackGQA与NumSplits的协同舞蹈"), so every KV byte crosses HBM once.
+// Scores and P·V run on warp-level tensor cores (m16n8k16, fp32 accumulate) with the
+// tile's tokens as M and the packed heads as N; the softmax is the online (running max /
+// running sum) form in fp32, exp2 domain, as in the tiled fused attention of
+// "TensorRT-LLM与TensorRT核心差异解析", section 4.2.1 FlashAttention.
 //
-// Warp roles: warp 4 is the producer (page-table resolve, TMA issue, one elected lane);
-// warps 0..3 are consumers, taking tiles round-robin, each with its own softmax state,
-// merged through shared memory at the end.  Every wait is bounded (2 s): on expiry the
-// kernel records GQA_ERR_TIMEOUT in the workspace error word and returns.
+// Warp roles: warp 4 is the producer (page-table resolve, TMA issue by one lane); warps
+// 0..3 are consumers.  Two schedules share the per-tile code (WarpAttn):
+//   - split (decode_kernel): one CTA per (split, kv head [, head chunk], sequence); the
+//     split's tiles go round-robin to the 4 warps, merged through shared memory at the
+//     end; splits (NumSplits) are merged by lse_combine.
+//   - balanced persistent (decode_sk_kernel): a fixed grid; all (sequence, kv head)
+//     tiles are laid end to end and every consumer warp takes an equal contiguous share.
+//     A warp that holds a whole (sequence, kv head) unit writes its output directly; a
+//     unit cut between warps leaves one piece per warp, and the last warp to finish its
+//     piece merges them by log-sum-exp (no second launch).
+// Every wait is bounded (2 s): on expiry the kernel records GQA_ERR_TIMEOUT in the
+// workspace error word and returns.
 //
 // Tile layout in shared memory (per K or V tile, 16 token rows): the row is cut into
 // 128-byte boxes (2 for bf16 D=128, 1 for bf16 D=64 and fp8 D=128); box j of row r sits
@@ -25,14 +33,19 @@
 namespace gqa {
 namespace {
 
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = kStreamWorkersPerCta;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kTile = kDecodeTileTokens;  // tokens per pipeline stage
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D, bool FP8>
+// Ring sizes: the split kernel runs 3 CTAs per SM with a 64 KB ring; the balanced
+// kernel runs 2 per SM (more registers per thread) with a 96 KB ring.
+constexpr int kRingSplit = 65536;
+constexpr int kRingBalanced = 98304;
+
+template <int D, bool FP8, int RING = kRingSplit>
 struct Cfg {
     static constexpr int kElt = FP8 ? 1 : 2;
     static constexpr int kRowBytes = D * kElt;
@@ -40,17 +53,29 @@ struct Cfg {
     static constexpr int kBoxCols = 128 / kElt;        // elements per box row
     static constexpr int kTileBytes = kTile * kRowBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kStagesRaw = 65536 / kStageBytes;
-    static constexpr int kStages = kStagesRaw < 4 ? 4 : (kStagesRaw > 16 ? 16 : kStagesRaw);
+    static constexpr int kStagesRaw = RING / kStageBytes;
+    static constexpr int kStages = kStagesRaw < 4 ? 4 : (kStagesRaw > 32 ? 32 : kStagesRaw);
+    static_assert(kStages % kConsumerWarps == 0, "stage i belongs to consumer warp i % 4");
 };
 
-template <int D, bool FP8>
+// Per-stage tile description written by the producer (balanced schedule).
+struct TileRec {
+    int b;       // sequence, or -1 for an empty slot
+    int y;       // unit within the sequence: kv head * head chunks + chunk
+    int tile;    // tile index within the unit
+    int valid;   // tokens of the tile inside the sequence
+    long long f; // flat tile index
+};
+
+template <int D, bool FP8, int RING = kRingSplit>
 struct alignas(1024) Smem {
-    uint8_t tiles[Cfg<D, FP8>::kStages][2][Cfg<D, FP8>::kTileBytes];
-    uint64_t full[Cfg<D, FP8>::kStages];
-    uint64_t empty[Cfg<D, FP8>::kStages];
-    float kscale[Cfg<D, FP8>::kStages];
-    float vscale[Cfg<D, FP8>::kStages];
+    using C = Cfg<D, FP8, RING>;
+    uint8_t tiles[C::kStages][2][C::kTileBytes];
+    uint64_t full[C::kStages];
+    uint64_t empty[C::kStages];
+    float kscale[C::kStages];
+    float vscale[C::kStages];
+    TileRec rec[C::kStages];
     int abort_flag;
 };
 
@@ -63,13 +88,263 @@ __device__ __forceinline__ void consumer_bar() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
+__device__ __forceinline__ int clamp_len(int L, int Lmax, int *err) {
+    if (L < 0 || L > Lmax) {
+        set_error(err, GQA_ERR_BAD_PAGE);
+        return L < 0 ? 0 : Lmax;
+    }
+    return L;
+}
+
+// One consumer warp's attention state for up to 8*NT packed heads of one kv head:
+// q fragments, the running max / sum per head, and O^T accumulators.
+//   fragment lane (gq = lane / 4, cq = lane % 4) holds heads 8*nt + 2*cq (+1) and, for
+//   dim tile dt, dims dim0(dt) and dim1(dt).
 template <int D, int NT, bool FP8>
-__global__ void __launch_bounds__(kThreads, 3)
+struct WarpAttn {
+    static constexpr int KT = D / 16;
+    uint32_t qf[NT][KT][2];
+    float qmul;  // fp8 path: power-of-two prescale bringing q into f16 range
+    float o[NT][KT][4];
+    float m[NT][2], l[NT][2];
+
+    __device__ __forceinline__ static int dim0(int dt, int gq) {
+        return FP8 ? dt * 16 + 4 * (gq >> 1) + (gq & 1) : dt * 16 + gq;
+    }
+    __device__ __forceinline__ static int dim1(int dt, int gq) {
+        return FP8 ? dim0(dt, gq) + 2 : dim0(dt, gq) + 8;
+    }
+
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int dt = 0; dt < KT; ++dt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[nt][dt][e] = 0.f;
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+        }
+    }
+
+    // q rows of the nh packed heads start at q_rows (row stride D).
+    __device__ __forceinline__ void load_q(const __nv_bfloat16 *q_rows, int nh, int lane) {
+        const int gq = lane >> 2, cq = lane & 3;
+        qmul = 1.f;
+        if (!FP8) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int hl = nt * 8 + gq;
+                const bool ok = hl < nh;
+                const uint32_t *qw = reinterpret_cast<const uint32_t *>(q_rows + (size_t)(ok ? hl : 0) * D);
+#pragma unroll
+                for (int ks = 0; ks < KT; ++ks) {
+                    qf[nt][ks][0] = ok ? __ldg(qw + (ks * 16 + 2 * cq) / 2) : 0u;
+                    qf[nt][ks][1] = ok ? __ldg(qw + (ks * 16 + 8 + 2 * cq) / 2) : 0u;
+                }
+            }
+        } else {
+            float qv[NT][KT][4];
+            float amax = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int hl = nt * 8 + gq;
+                const bool ok = hl < nh;
+                const uint2 *qw = reinterpret_cast<const uint2 *>(q_rows + (size_t)(ok ? hl : 0) * D);
+#pragma unroll
+                for (int ks = 0; ks < KT; ++ks) {
+                    uint2 w = ok ? __ldg(qw + (ks * 16 + 4 * cq) / 4) : make_uint2(0u, 0u);
+                    __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162 *>(&w.x);
+                    __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162 *>(&w.y);
+                    qv[nt][ks][0] = __low2float(lo);
+                    qv[nt][ks][1] = __high2float(lo);
+                    qv[nt][ks][2] = __low2float(hi);
+                    qv[nt][ks][3] = __high2float(hi);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[nt][ks][e]));
+                }
+            }
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o2));
+            if (amax > 0.f && amax < 3.0e38f) {
+                int e;
+                frexpf(amax, &e);  // amax < 2^e
+                qmul = ldexpf(1.f, min(126, 15 - e));
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int ks = 0; ks < KT; ++ks) {
+                    qf[nt][ks][0] = pack_f16(qv[nt][ks][0] * qmul, qv[nt][ks][1] * qmul);
+                    qf[nt][ks][1] = pack_f16(qv[nt][ks][2] * qmul, qv[nt][ks][3] * qmul);
+                }
+        }
+    }
+
+    // Fold one 16-token tile (valid tokens first, rows past them ignored) into the state.
+    __device__ __forceinline__ void tile(uint8_t *kt, uint8_t *vt, int valid, float scale_log2,
+                                         float ksc, float vsc, int lane) {
+        using C = Cfg<D, FP8>;
+        const int gq = lane >> 2;
+        if (valid < kTile) {
+            // Rows past the end of the sequence may hold anything (even NaN): zero the V
+            // rows so 0-weight tokens contribute exactly 0; K rows are masked below.
+            constexpr int kChunksPerRow = C::kRowBytes / 16;
+            for (int e = lane; e < (kTile - valid) * kChunksPerRow; e += 32) {
+                const int r = valid + e / kChunksPerRow, cb = (e % kChunksPerRow) * 16;
+                *reinterpret_cast<uint4 *>(vt + swz(r, cb)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
+        const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
+
+        // ---- scores S^T[token][head] = K q^T
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        if (!FP8) {
+            const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int ks = 0; ks < KT; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(af, kbase + swz(r, (ks * 16 + (lane >> 4) * 8) * 2));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(s[nt], af, qf[nt][ks][0], qf[nt][ks][1]);
+            }
+        } else {
+            // One ldmatrix.x4 over 32 fp8 dims serves two k steps; the k order inside a
+            // step is permuted identically for K (here) and q (qf), which leaves each dot
+            // product unchanged.
+            const int j = lane >> 3;
+            const int r = (lane & 7) + (j & 1) * 8;
+#pragma unroll
+            for (int kp = 0; kp < D / 32; ++kp) {
+                uint32_t raw[4];
+                ldsm_x4(raw, kbase + swz(r, 32 * kp + (j >> 1) * 16));
+                uint32_t a0[4] = {e4m3x2_to_f16x2(raw[0] & 0xffff), e4m3x2_to_f16x2(raw[1] & 0xffff),
+                                  e4m3x2_to_f16x2(raw[0] >> 16), e4m3x2_to_f16x2(raw[1] >> 16)};
+                uint32_t a1[4] = {e4m3x2_to_f16x2(raw[2] & 0xffff), e4m3x2_to_f16x2(raw[3] & 0xffff),
+                                  e4m3x2_to_f16x2(raw[2] >> 16), e4m3x2_to_f16x2(raw[3] >> 16)};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_f16(s[nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+                    mma_f16(s[nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                }
+            }
+        }
+
+        // ---- online softmax (exp2 domain), per packed head column
+        const float kmul = FP8 ? scale_log2 * ksc / qmul : scale_log2;
+        const bool v0 = gq < valid, v1 = gq + 8 < valid;
+        uint32_t pb[NT][2], pbl[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float p[4], alpha[2];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const float x0 = v0 ? s[nt][jj] * kmul : -INFINITY;
+                const float x1 = v1 ? s[nt][jj + 2] * kmul : -INFINITY;
+                float mx = fmaxf(x0, x1);
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+                const float mnew = fmaxf(m[nt][jj], mx);
+                const float mref = mnew == -INFINITY ? 0.f : mnew;
+                alpha[jj] = fast_exp2(m[nt][jj] - mref);
+                p[jj] = fast_exp2(x0 - mref);
+                p[jj + 2] = fast_exp2(x1 - mref);
+                l[nt][jj] = l[nt][jj] * alpha[jj] + p[jj] + p[jj + 2];
+                m[nt][jj] = mnew;
+            }
+            if (!FP8) {
+                // P as a bf16 value plus its bf16 residual: O += V^T P_hi^T + V^T P_lo^T keeps
+                // the weights at ~16 bits (one bf16 P would cost up to 2^-9 per weight).
+                uint32_t h0, l0, h1, l1;
+                split_bf16x2(p[0], p[1], h0, l0);
+                split_bf16x2(p[2], p[3], h1, l1);
+                pb[nt][0] = movmatrix_trans(h0);
+                pb[nt][1] = movmatrix_trans(h1);
+                pbl[nt][0] = movmatrix_trans(l0);
+                pbl[nt][1] = movmatrix_trans(l1);
+            } else {
+                pb[nt][0] = movmatrix_trans(pack_f16(p[0], p[1]));
+                pb[nt][1] = movmatrix_trans(pack_f16(p[2], p[3]));
+            }
+#pragma unroll
+            for (int dt = 0; dt < KT; ++dt) {
+                o[nt][dt][0] *= alpha[0];
+                o[nt][dt][1] *= alpha[1];
+                o[nt][dt][2] *= alpha[0];
+                o[nt][dt][3] *= alpha[1];
+            }
+        }
+
+        // ---- O^T[dim][head] += V^T P^T
+        if (!FP8) {
+            const int j = lane >> 3;
+            const int r = (lane & 7) + (j >> 1) * 8;
+#pragma unroll
+            for (int dt = 0; dt < KT; ++dt) {
+                uint32_t af[4];
+                ldsm_x4_trans(af, vbase + swz(r, (dt * 16 + (j & 1) * 8) * 2));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16(o[nt][dt], af, pb[nt][0], pb[nt][1]);
+                    mma_bf16(o[nt][dt], af, pbl[nt][0], pbl[nt][1]);
+                }
+            }
+        } else {
+            // fp8 V: plain ldmatrix gives each lane 4 consecutive dims of one token;
+            // after conversion, movmatrix transposes 8x8 blocks into the A layout (dims
+            // permuted within each 16-dim tile; dim0/dim1 undo it when O is written).
+            const int j = lane >> 3;
+            const int r = (lane & 7) + (j & 1) * 8;
+#pragma unroll
+            for (int qd = 0; qd < D / 32; ++qd) {
+                uint32_t raw[4];
+                ldsm_x4(raw, vbase + swz(r, 32 * qd + (j >> 1) * 16));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t lo_t = raw[2 * h], hi_t = raw[2 * h + 1];  // tokens 0-7 / 8-15
+                    uint32_t af[4] = {movmatrix_trans(e4m3x2_to_f16x2(lo_t & 0xffff)),
+                                      movmatrix_trans(e4m3x2_to_f16x2(lo_t >> 16)),
+                                      movmatrix_trans(e4m3x2_to_f16x2(hi_t & 0xffff)),
+                                      movmatrix_trans(e4m3x2_to_f16x2(hi_t >> 16))};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float pv[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_f16(pv, af, pb[nt][0], pb[nt][1]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[nt][2 * qd + h][e] += vsc * pv[e];
+                    }
+                }
+            }
+        }
+    }
+
+    // Sum the per-lane partial sums l over the 8 lanes sharing a head column.
+    __device__ __forceinline__ void finish_l() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                float v = l[nt][jj];
+                v += __shfl_xor_sync(kFull, v, 4);
+                v += __shfl_xor_sync(kFull, v, 8);
+                v += __shfl_xor_sync(kFull, v, 16);
+                l[nt][jj] = v;
+            }
+    }
+};
+
+// ========================================================================== split schedule
+template <int D, int NT, bool FP8>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const DecodeArgs a, const int heads_per_cta, const int head_chunks) {
     using C = Cfg<D, FP8>;
     constexpr int S = C::kStages;
-    constexpr int KT = D / 16;  // 16-wide k steps (scores) and dim tiles (output)
+    constexpr int KT = D / 16;
     extern __shared__ uint8_t smem_raw[];
     Smem<D, FP8> &sm = *reinterpret_cast<Smem<D, FP8> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -85,12 +360,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 
     // This split's token range [t0, t1), page aligned (contiguous ranges of
     // ceil(np / num_splits) pages).
-    int L = a.seq_lens[b];
-    const int Lmax = a.pt_stride * P;
-    if (L < 0 || L > Lmax) {
-        if (threadIdx.x == 0) set_error(a.err, GQA_ERR_BAD_PAGE);
-        L = L < 0 ? 0 : Lmax;
-    }
+    const int L = clamp_len(a.seq_lens[b], a.pt_stride * P, threadIdx.x == 0 ? a.err : nullptr);
     const int np = (L + P - 1) / P;
     const int cpp = (np + a.num_splits - 1) / a.num_splits;
     const int t0 = split * cpp * P;
@@ -179,76 +449,10 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
 
     // -------------------------------------------------------------------- consumers
-    const int gq = lane >> 2, cq = lane & 3;  // fragment row group / column pair
-
-    // q as the B operand (k = head dim, n = packed head), registers for the whole CTA.
-    uint32_t qf[NT][KT][2];
-    float qmul = 1.f;  // fp8 path: power-of-two prescale bringing q into f16 range
-    {
-        const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-        if (!FP8) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int hl = nt * 8 + gq;
-                const bool ok = hl < nh;
-                const uint32_t *qw = reinterpret_cast<const uint32_t *>(
-                    qb + ((size_t)b * a.Hq + head_lo + (ok ? hl : 0)) * D);
-#pragma unroll
-                for (int ks = 0; ks < KT; ++ks) {
-                    qf[nt][ks][0] = ok ? __ldg(qw + (ks * 16 + 2 * cq) / 2) : 0u;
-                    qf[nt][ks][1] = ok ? __ldg(qw + (ks * 16 + 8 + 2 * cq) / 2) : 0u;
-                }
-            }
-        } else {
-            float qv[NT][KT][4];
-            float amax = 0.f;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int hl = nt * 8 + gq;
-                const bool ok = hl < nh;
-                const uint2 *qw = reinterpret_cast<const uint2 *>(
-                    qb + ((size_t)b * a.Hq + head_lo + (ok ? hl : 0)) * D);
-#pragma unroll
-                for (int ks = 0; ks < KT; ++ks) {
-                    uint2 w = ok ? __ldg(qw + (ks * 16 + 4 * cq) / 4) : make_uint2(0u, 0u);
-                    __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162 *>(&w.x);
-                    __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162 *>(&w.y);
-                    qv[nt][ks][0] = __low2float(lo);
-                    qv[nt][ks][1] = __high2float(lo);
-                    qv[nt][ks][2] = __low2float(hi);
-                    qv[nt][ks][3] = __high2float(hi);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[nt][ks][e]));
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-            if (amax > 0.f && amax < 3.0e38f) {
-                int e;
-                frexpf(amax, &e);  // amax < 2^e
-                qmul = ldexpf(1.f, min(126, 15 - e));
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int ks = 0; ks < KT; ++ks) {
-                    qf[nt][ks][0] = pack_f16(qv[nt][ks][0] * qmul, qv[nt][ks][1] * qmul);
-                    qf[nt][ks][1] = pack_f16(qv[nt][ks][2] * qmul, qv[nt][ks][3] * qmul);
-                }
-        }
-    }
-
-    float o[NT][KT][4];
-    float m[NT][2], l[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int dt = 0; dt < KT; ++dt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[nt][dt][e] = 0.f;
-        m[nt][0] = m[nt][1] = -INFINITY;
-        l[nt][0] = l[nt][1] = 0.f;
-    }
+    const int gq = lane >> 2, cq = lane & 3;
+    WarpAttn<D, NT, FP8> st;
+    st.load_q(reinterpret_cast<const __nv_bfloat16 *>(a.q) + ((size_t)b * a.Hq + head_lo) * D, nh, lane);
+    st.reset();
     const float scale_log2 = a.scale * kLog2e;
 
     bool fail = false;
@@ -259,160 +463,14 @@ __global__ void __launch_bounds__(kThreads, 3)
             fail = true;
             break;
         }
-        uint8_t *kt = sm.tiles[stage][0];
-        uint8_t *vt = sm.tiles[stage][1];
-        const int valid = t1 - (t0 + it * kTile);  // >= 1
-        if (valid < kTile) {
-            // Rows past the end of the sequence may hold anything (even NaN): zero the V
-            // rows so 0-weight tokens contribute exactly 0; K rows are masked below.
-            constexpr int kChunksPerRow = C::kRowBytes / 16;
-            for (int e = lane; e < (kTile - valid) * kChunksPerRow; e += 32) {
-                const int r = valid + e / kChunksPerRow, cb = (e % kChunksPerRow) * 16;
-                *reinterpret_cast<uint4 *>(vt + swz(r, cb)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            __syncwarp();
-        }
-        const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
-
-        // ---- scores S^T[token][head] = K q^T
-        float s[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-        if (!FP8) {
-            const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int ks = 0; ks < KT; ++ks) {
-                uint32_t af[4];
-                ldsm_x4(af, kbase + swz(r, (ks * 16 + (lane >> 4) * 8) * 2));
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16(s[nt], af, qf[nt][ks][0], qf[nt][ks][1]);
-            }
-        } else {
-            // One ldmatrix.x4 over 32 fp8 dims serves two k steps; the k order inside a
-            // step is permuted identically for K (here) and q (qf), which leaves each dot
-            // product unchanged.
-            const int j = lane >> 3;
-            const int r = (lane & 7) + (j & 1) * 8;
-#pragma unroll
-            for (int kp = 0; kp < D / 32; ++kp) {
-                uint32_t raw[4];
-                ldsm_x4(raw, kbase + swz(r, 32 * kp + (j >> 1) * 16));
-                uint32_t a0[4] = {e4m3x2_to_f16x2(raw[0] & 0xffff), e4m3x2_to_f16x2(raw[1] & 0xffff),
-                                  e4m3x2_to_f16x2(raw[0] >> 16), e4m3x2_to_f16x2(raw[1] >> 16)};
-                uint32_t a1[4] = {e4m3x2_to_f16x2(raw[2] & 0xffff), e4m3x2_to_f16x2(raw[3] & 0xffff),
-                                  e4m3x2_to_f16x2(raw[2] >> 16), e4m3x2_to_f16x2(raw[3] >> 16)};
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_f16(s[nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-                    mma_f16(s[nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
-                }
-            }
-        }
-
-        // ---- online softmax (exp2 domain), per packed head column
-        const float kmul = FP8 ? scale_log2 * sm.kscale[stage] / qmul : scale_log2;
-        const bool v0 = gq < valid, v1 = gq + 8 < valid;
-        uint32_t pb[NT][2], pbl[NT][2];
-        float alpha[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float p[4];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const float x0 = v0 ? s[nt][jj] * kmul : -INFINITY;
-                const float x1 = v1 ? s[nt][jj + 2] * kmul : -INFINITY;
-                float mx = fmaxf(x0, x1);
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                const float mnew = fmaxf(m[nt][jj], mx);
-                const float mref = mnew == -INFINITY ? 0.f : mnew;
-                alpha[nt][jj] = fast_exp2(m[nt][jj] - mref);
-                p[jj] = fast_exp2(x0 - mref);
-                p[jj + 2] = fast_exp2(x1 - mref);
-                l[nt][jj] = l[nt][jj] * alpha[nt][jj] + p[jj] + p[jj + 2];
-                m[nt][jj] = mnew;
-            }
-            if (!FP8) {
-                // P as a bf16 value plus its bf16 residual: O += V^T P_hi^T + V^T P_lo^T keeps
-                // the weights at ~16 bits (one bf16 P would cost up to 2^-9 per weight).
-                uint32_t h0, l0, h1, l1;
-                split_bf16x2(p[0], p[1], h0, l0);
-                split_bf16x2(p[2], p[3], h1, l1);
-                pb[nt][0] = movmatrix_trans(h0);
-                pb[nt][1] = movmatrix_trans(h1);
-                pbl[nt][0] = movmatrix_trans(l0);
-                pbl[nt][1] = movmatrix_trans(l1);
-            } else {
-                pb[nt][0] = movmatrix_trans(pack_f16(p[0], p[1]));
-                pb[nt][1] = movmatrix_trans(pack_f16(p[2], p[3]));
-            }
-#pragma unroll
-            for (int dt = 0; dt < KT; ++dt) {
-                o[nt][dt][0] *= alpha[nt][0];
-                o[nt][dt][1] *= alpha[nt][1];
-                o[nt][dt][2] *= alpha[nt][0];
-                o[nt][dt][3] *= alpha[nt][1];
-            }
-        }
-
-        // ---- O^T[dim][head] += V^T P^T
-        if (!FP8) {
-            const int j = lane >> 3;
-            const int r = (lane & 7) + (j >> 1) * 8;
-#pragma unroll
-            for (int dt = 0; dt < KT; ++dt) {
-                uint32_t af[4];
-                ldsm_x4_trans(af, vbase + swz(r, (dt * 16 + (j & 1) * 8) * 2));
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_bf16(o[nt][dt], af, pb[nt][0], pb[nt][1]);
-                    mma_bf16(o[nt][dt], af, pbl[nt][0], pbl[nt][1]);
-                }
-            }
-        } else {
-            // fp8 V: plain ldmatrix gives each lane 4 consecutive dims of one token;
-            // after conversion, movmatrix transposes 8x8 blocks into the A layout (dims
-            // permuted within each 16-dim tile, undone when O is written out).
-            const float vsc = sm.vscale[stage];
-            const int j = lane >> 3;
-            const int r = (lane & 7) + (j & 1) * 8;
-#pragma unroll
-            for (int qd = 0; qd < D / 32; ++qd) {
-                uint32_t raw[4];
-                ldsm_x4(raw, vbase + swz(r, 32 * qd + (j >> 1) * 16));
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t lo_t = raw[2 * h], hi_t = raw[2 * h + 1];  // tokens 0-7 / 8-15
-                    uint32_t af[4] = {movmatrix_trans(e4m3x2_to_f16x2(lo_t & 0xffff)),
-                                      movmatrix_trans(e4m3x2_to_f16x2(lo_t >> 16)),
-                                      movmatrix_trans(e4m3x2_to_f16x2(hi_t & 0xffff)),
-                                      movmatrix_trans(e4m3x2_to_f16x2(hi_t >> 16))};
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        float pv[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_f16(pv, af, pb[nt][0], pb[nt][1]);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) o[nt][2 * qd + h][e] += vsc * pv[e];
-                    }
-                }
-            }
-        }
+        st.tile(sm.tiles[stage][0], sm.tiles[stage][1], t1 - (t0 + it * kTile), scale_log2,
+                FP8 ? sm.kscale[stage] : 1.f, FP8 ? sm.vscale[stage] : 1.f, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[stage]);
     }
 
     // ------------------------------------------------------------------ epilogue
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-            float v = l[nt][jj];
-            v += __shfl_xor_sync(kFull, v, 4);
-            v += __shfl_xor_sync(kFull, v, 8);
-            v += __shfl_xor_sync(kFull, v, 16);
-            l[nt][jj] = v;
-        }
+    st.finish_l();
     if (fail && lane == 0) {
         set_error(a.err, GQA_ERR_TIMEOUT);
         sm.abort_flag = 1;
@@ -430,25 +488,18 @@ __global__ void __launch_bounds__(kThreads, 3)
         const int h0 = nt * 8 + 2 * cq;
 #pragma unroll
         for (int dt = 0; dt < KT; ++dt) {
-            int d0, d1;
-            if (!FP8) {
-                d0 = dt * 16 + gq;
-                d1 = d0 + 8;
-            } else {
-                d0 = dt * 16 + 4 * (gq >> 1) + (gq & 1);
-                d1 = d0 + 2;
-            }
+            const int d0 = WarpAttn<D, NT, FP8>::dim0(dt, gq), d1 = WarpAttn<D, NT, FP8>::dim1(dt, gq);
             float *w = red_o + (size_t)(warp * HW + h0) * RS;
-            w[d0] = o[nt][dt][0];
-            w[RS + d0] = o[nt][dt][1];
-            w[d1] = o[nt][dt][2];
-            w[RS + d1] = o[nt][dt][3];
+            w[d0] = st.o[nt][dt][0];
+            w[RS + d0] = st.o[nt][dt][1];
+            w[d1] = st.o[nt][dt][2];
+            w[RS + d1] = st.o[nt][dt][3];
         }
         if (gq == 0) {
-            red_m[warp * HW + h0] = m[nt][0];
-            red_m[warp * HW + h0 + 1] = m[nt][1];
-            red_l[warp * HW + h0] = l[nt][0];
-            red_l[warp * HW + h0 + 1] = l[nt][1];
+            red_m[warp * HW + h0] = st.m[nt][0];
+            red_m[warp * HW + h0 + 1] = st.m[nt][1];
+            red_l[warp * HW + h0] = st.l[nt][0];
+            red_l[warp * HW + h0 + 1] = st.l[nt][1];
         }
     }
     consumer_bar();
@@ -484,19 +535,366 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
 }
 
+// ========================================================== balanced persistent schedule
+//
+// Flat tile space: sequence b owns tiles [U*pre[b], U*pre[b+1]) with pre[] the prefix of
+// nt_b = ceil(L_b / 16) and U = Hk * head chunks units per sequence; unit y of sequence
+// b owns [U*pre[b] + y*nt_b, ... + nt_b).  With T tiles and NW workers (at most one per
+// kMinTilesPerWorker tiles), worker W owns [W*T/NW, (W+1)*T/NW) (floor divisions): every
+// worker gets one tile more or less than any other.
+//
+// Each consumer warp is one worker with a private sub-ring of S/4 stages fed by its own
+// producer lane (lane w of warp 4), so a warp that pauses (loading the next unit's q,
+// merging pieces) never holds up the other warps' streams.
+
+constexpr int kMinTilesPerWorker = 16;
+
+__device__ __forceinline__ long long sk_start(long long W, long long T, long long NW) {
+    return W >= NW ? T : (W * T) / NW;
+}
+// The worker whose range holds flat tile t: max W with sk_start(W) <= t.
+__device__ __forceinline__ long long sk_worker_of(long long t, long long T, long long NW) {
+    return ((t + 1) * NW + T - 1) / T - 1;
+}
+
+// Position (sequence, unit, tile) of flat tile f, and a step to the next flat tile.
+struct FlatPos {
+    int b, y, tile, nt;
+};
+
+__device__ __forceinline__ FlatPos flat_locate(long long f, const int *pre, int B, int U) {
+    int lo = 0, hi = B - 1;  // smallest b with U*pre[b+1] > f
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)U * pre[mid + 1] > f) hi = mid; else lo = mid + 1;
+    }
+    FlatPos p;
+    p.b = lo;
+    p.nt = pre[lo + 1] - pre[lo];
+    const long long local = f - (long long)U * pre[lo];
+    p.y = (int)(local / p.nt);
+    p.tile = (int)(local % p.nt);
+    return p;
+}
+
+__device__ __forceinline__ void flat_next(FlatPos &p, const int *pre, int U) {
+    if (++p.tile < p.nt) return;
+    p.tile = 0;
+    if (++p.y < U) return;
+    p.y = 0;
+    do {
+        ++p.b;
+        p.nt = pre[p.b + 1] - pre[p.b];
+    } while (p.nt == 0);
+}
+
+// Merge of every piece of one unit (pieces of workers wfirst..wlast; side 1 for the
+// first, side 0 for the rest) by one online log-sum-exp pass.  Lane owns dims
+// [DV*lane, DV*lane + DV) of every head; each piece's loads are independent of each
+// other.  Kept out of line: it runs once per shared unit and its arrays would otherwise
+// crowd the streaming loop's registers.
+template <int D, int HW>
+__device__ __forceinline__ void merge_pieces(const float *pieces, long long wfirst, long long wlast,
+                                          int slot_floats, int hpc, int nh, __nv_bfloat16 *out_rows,
+                                          float *lse_rows, int lane) {
+    constexpr int DV = D / 32;
+    float Mh[HW], Wh[HW], acc[HW][DV];
+#pragma unroll
+    for (int h = 0; h < HW; ++h) {
+        Mh[h] = -INFINITY;
+        Wh[h] = 0.f;
+#pragma unroll
+        for (int v = 0; v < DV; ++v) acc[h][v] = 0.f;
+    }
+    for (long long W = wfirst; W <= wlast; ++W) {
+        const float *ps = pieces + (size_t)(W * 2 + (W == wfirst ? 1 : 0)) * slot_floats;
+        float lv[HW], ov[HW][DV];
+#pragma unroll
+        for (int h = 0; h < HW; ++h) {
+            if (h < nh) {
+                lv[h] = __ldcg(ps + hpc * D + h);
+                if constexpr (DV == 4) {
+                    const float4 t = __ldcg(reinterpret_cast<const float4 *>(ps + h * D + DV * lane));
+                    ov[h][0] = t.x; ov[h][1] = t.y; ov[h][2] = t.z; ov[h][3] = t.w;
+                } else {
+                    const float2 t = __ldcg(reinterpret_cast<const float2 *>(ps + h * D + DV * lane));
+                    ov[h][0] = t.x; ov[h][1] = t.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < HW; ++h) {
+            if (h >= nh) continue;
+            const float mnew = fmaxf(Mh[h], lv[h]);
+            const float c_old = __expf(Mh[h] - mnew), c_new = __expf(lv[h] - mnew);
+            Wh[h] = Wh[h] * c_old + c_new;
+#pragma unroll
+            for (int v = 0; v < DV; ++v) acc[h][v] = acc[h][v] * c_old + c_new * ov[h][v];
+            Mh[h] = mnew;
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < HW; ++h) {
+        if (h >= nh) continue;
+        const float inv = 1.f / Wh[h];
+        __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(out_rows + (size_t)h * D + DV * lane);
+#pragma unroll
+        for (int v = 0; v < DV; v += 2) dst[v / 2] = __floats2bfloat162_rn(acc[h][v] * inv, acc[h][v + 1] * inv);
+        if (lane == 0 && lse_rows) lse_rows[h] = Mh[h] + logf(Wh[h]);
+    }
+}
+
+template <int D, int NT, bool FP8>
+__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
+    decode_sk_kernel(const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, const DecodeArgs a,
+                     const int heads_per_cta, const int head_chunks) {
+    using C = Cfg<D, FP8, kRingBalanced>;
+    using SM = Smem<D, FP8, kRingBalanced>;
+    using WA = WarpAttn<D, NT, FP8>;
+    constexpr int S = C::kStages;
+    constexpr int SW = S / kConsumerWarps;  // stages per worker
+    constexpr int KT = D / 16;
+    constexpr int HW = 8 * NT;               // packed head columns
+    extern __shared__ uint8_t smem_raw[];
+    SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    int *pre = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(&sm) + sizeof(SM));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = a.B, P = a.P, g = a.Hq / a.Hk;
+    const int U = a.Hk * head_chunks;
+    const int Lmax = a.pt_stride * P;
+
+    // Tiles per sequence and their exclusive prefix (warp 0; lane i owns a run of sequences).
+    if (warp == 0) {
+        const int per = (B + 31) / 32;
+        const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
+        int sum = 0;
+        for (int b = b0; b < b1; ++b)
+            sum += (clamp_len(a.seq_lens[b], Lmax, blockIdx.x == 0 ? a.err : nullptr) + kTile - 1) / kTile;
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int run = incl - sum;
+        for (int b = b0; b < b1; ++b) {
+            pre[b] = run;
+            run += (clamp_len(a.seq_lens[b], Lmax, nullptr) + kTile - 1) / kTile;
+        }
+        if (lane == 31) pre[B] = incl;
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        sm.abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    const long long T = (long long)U * pre[B];
+    const long long NW = min((long long)gridDim.x * kConsumerWarps,
+                             max(1LL, T / kMinTilesPerWorker));
+    const long long W0cta = (long long)blockIdx.x * kConsumerWarps;
+
+    // Sequences with no tokens have no tiles: their outputs are written here (zeros, -inf).
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
+        if (pre[b + 1] != pre[b]) continue;
+        __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(a.out) + (size_t)b * a.Hq * D;
+        for (int e = threadIdx.x; e < a.Hq * D; e += kThreads) ob[e] = __float2bfloat16(0.f);
+        if (a.lse)
+            for (int e = threadIdx.x; e < a.Hq; e += kThreads) a.lse[(size_t)b * a.Hq + e] = -INFINITY;
+    }
+    if (T == 0) return;
+
+    if (warp == kConsumerWarps) {
+        // ---------------------------------------------- producer: lane w feeds worker w
+        if (lane >= kConsumerWarps) return;
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+        }
+        const uint64_t pol = a.pack_gqa ? policy_evict_first() : policy_evict_last();
+        const long long s_w = sk_start(W0cta + lane, T, NW), e_w = sk_start(W0cta + lane + 1, T, NW);
+        const long long n = e_w - s_w;
+        long long issued = 0;
+        FlatPos pos;
+        if (n > 0) pos = flat_locate(s_w, pre, B, U);
+        for (long long r = 0; r < n; ++r) {
+            if (r > 0) flat_next(pos, pre, U);
+            const int stage = lane * SW + (int)(r % SW);
+            const long long use = r / SW;
+            if (use > 0 && !mbar_wait(&sm.empty[stage], (uint32_t)((use - 1) & 1))) {
+                set_error(a.err, GQA_ERR_TIMEOUT);
+                break;
+            }
+            const int L = clamp_len(a.seq_lens[pos.b], Lmax, nullptr);
+            const int tok0 = pos.tile * kTile;
+            const int kvh = pos.y / head_chunks;
+            TileRec rec;
+            rec.b = pos.b;
+            rec.y = pos.y;
+            rec.tile = pos.tile;
+            rec.valid = min(kTile, L - tok0);
+            rec.f = s_w + r;
+            const int phys = __ldg(a.page_table + (size_t)pos.b * a.pt_stride + tok0 / P);
+            sm.rec[stage] = rec;
+            if (phys < 0 || phys >= a.num_pages) {
+                set_error(a.err, GQA_ERR_BAD_PAGE);
+                mbar_arrive(&sm.full[stage]);  // no copy: the tile computes on stale data
+            } else {
+                if (FP8) {
+                    sm.kscale[stage] = __ldg(a.k_scale + (size_t)phys * a.Hk + kvh);
+                    sm.vscale[stage] = __ldg(a.v_scale + (size_t)phys * a.Hk + kvh);
+                }
+                const int row = (phys * a.Hk + kvh) * P + tok0 % P;
+                mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
+#pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128, &kmap, &sm.full[stage],
+                                bx * C::kBoxCols, row, pol);
+                    tma_load_2d(sm.tiles[stage][1] + bx * kTile * 128, &vmap, &sm.full[stage],
+                                bx * C::kBoxCols, row, pol);
+                }
+            }
+            issued = r + 1;
+        }
+        // no copy into this CTA's shared memory may outlive it
+        for (long long r = max(0LL, issued - SW); r < issued; ++r)
+            if (!mbar_wait(&sm.full[lane * SW + (int)(r % SW)], (uint32_t)((r / SW) & 1))) {
+                set_error(a.err, GQA_ERR_TIMEOUT);
+                break;
+            }
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int gq = lane >> 2, cq = lane & 3;
+    const long long Wme = W0cta + warp;
+    const long long s_w = sk_start(Wme, T, NW), e_w = sk_start(Wme + 1, T, NW);
+    const long long n = e_w - s_w;
+    const float scale_log2 = a.scale * kLog2e;
+    // piece slot: heads_per_cta rows of D, then heads_per_cta lse values, padded to a
+    // multiple of 4 floats so every slot (and row) starts 16-byte aligned for the merge
+    const int slot_floats = (heads_per_cta * (D + 1) + 3) & ~3;
+    WA st;
+    st.reset();
+    st.qmul = 1.f;
+    int cur_b = -1, cur_y = -1;
+    for (long long r = 0; r < n; ++r) {
+        const int stage = warp * SW + (int)(r % SW);
+        const bool ok = mbar_wait(&sm.full[stage], (uint32_t)((r / SW) & 1));
+        if (__any_sync(kFull, !ok)) {
+            if (lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
+            break;
+        }
+        const TileRec rec = sm.rec[stage];
+        const float ks = FP8 ? sm.kscale[stage] : 1.f, vs = FP8 ? sm.vscale[stage] : 1.f;
+        const int b = rec.b, y = rec.y;
+        const int kvh = y / head_chunks, chunk = y % head_chunks;
+        const int head_lo = kvh * g + chunk * heads_per_cta;
+        const int nh = min(heads_per_cta, g - chunk * heads_per_cta);
+        if (b != cur_b || y != cur_y) {
+            st.reset();
+            st.load_q(reinterpret_cast<const __nv_bfloat16 *>(a.q) + ((size_t)b * a.Hq + head_lo) * D,
+                      nh, lane);
+            cur_b = b;
+            cur_y = y;
+        }
+        st.tile(sm.tiles[stage][0], sm.tiles[stage][1], rec.valid, scale_log2, ks, vs, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        const int nt_b = pre[b + 1] - pre[b];
+        if (rec.tile != nt_b - 1 && rec.f != e_w - 1) continue;
+
+        // ---- this warp's share of unit (b, y) is done
+        st.finish_l();
+        const long long us = (long long)U * pre[b] + (long long)y * nt_b, ue = us + nt_b;
+        const size_t row0 = (size_t)b * a.Hq + head_lo;
+        if (us >= s_w && ue <= e_w) {
+            // the whole unit: write the output directly
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int h = nt * 8 + 2 * cq + jj;
+                    if (h >= nh) continue;
+                    const float inv = st.l[nt][jj] > 0.f ? 1.f / st.l[nt][jj] : 0.f;
+                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) + (row0 + h) * D;
+#pragma unroll
+                    for (int dt = 0; dt < KT; ++dt) {
+                        dst[WA::dim0(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj] * inv);
+                        dst[WA::dim1(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj + 2] * inv);
+                    }
+                    if (gq == 0 && a.lse)
+                        a.lse[row0 + h] = st.l[nt][jj] > 0.f
+                                              ? (st.m[nt][jj] + __log2f(st.l[nt][jj])) * kLn2
+                                              : -INFINITY;
+                }
+        } else {
+            // a piece of a unit shared with neighbouring workers: side 0 = the unit began
+            // before this worker's range, side 1 = it begins here and continues after.
+            const int side = us < s_w ? 0 : 1;
+            float *slot = a.pieces + (size_t)(Wme * 2 + side) * slot_floats;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int h = nt * 8 + 2 * cq + jj;
+                    if (h >= nh) continue;
+                    const float inv = 1.f / st.l[nt][jj];
+#pragma unroll
+                    for (int dt = 0; dt < KT; ++dt) {
+                        slot[h * D + WA::dim0(dt, gq)] = st.o[nt][dt][jj] * inv;
+                        slot[h * D + WA::dim1(dt, gq)] = st.o[nt][dt][jj + 2] * inv;
+                    }
+                    if (gq == 0) slot[heads_per_cta * D + h] = (st.m[nt][jj] + __log2f(st.l[nt][jj])) * kLn2;
+                }
+            __threadfence();
+            __syncwarp();
+            const long long wfirst = sk_worker_of(us, T, NW), wlast = sk_worker_of(ue - 1, T, NW);
+            const int npieces = (int)(wlast - wfirst + 1);
+            int last = 0;
+            if (lane == 0) last = atomicAdd(a.counters + (size_t)b * U + y, 1) == npieces - 1;
+            last = __shfl_sync(kFull, last, 0);
+            if (last) {
+                __threadfence();
+                merge_pieces<D, HW>(a.pieces, wfirst, wlast, slot_floats, heads_per_cta, nh,
+                                    reinterpret_cast<__nv_bfloat16 *>(a.out) + row0 * D,
+                                    a.lse ? a.lse + row0 : nullptr, lane);
+                if (lane == 0) a.counters[(size_t)b * U + y] = 0;  // ready for the next launch
+            }
+        }
+        st.reset();
+        cur_b = -1;
+    }
+}
+
 template <int D, int NT, bool FP8>
 cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
-    const size_t smem = sizeof(Smem<D, FP8>) + 1024;
     static_assert(sizeof(float) * kConsumerWarps * 8 * NT * (D + 6) <=
                       sizeof(uint8_t) * Cfg<D, FP8>::kStages * 2 * Cfg<D, FP8>::kTileBytes,
                   "reduction area must fit in the stage ring");
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int g = a.Hq / a.Hk;
     const int hpc = a.pack_gqa ? (g < 8 * NT ? g : 8 * NT) : 1;
     const int chunks = (g + hpc - 1) / hpc;
+    if (a.stream_k) {
+        const size_t smem = sizeof(Smem<D, FP8, kRingBalanced>) + 1024 + sizeof(int) * (size_t)(a.B + 1);
+        cudaError_t e = cudaFuncSetAttribute(decode_sk_kernel<D, NT, FP8>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        decode_sk_kernel<D, NT, FP8><<<a.grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
+        return cudaGetLastError();
+    }
+    const size_t smem = sizeof(Smem<D, FP8>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     dim3 grid(a.num_splits, a.Hk * chunks, a.B);
     decode_kernel<D, NT, FP8><<<grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
     return cudaGetLastError();

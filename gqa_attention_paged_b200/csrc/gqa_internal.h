@@ -26,7 +26,26 @@ struct DecodeArgs {
     float *lse;
     float *o_part, *lse_part;  // scratch for num_splits > 1
     int *err;
+    // balanced persistent schedule (num_splits == 0, B <= kStreamMaxBatch)
+    int stream_k;
+    int *counters;  // [B * units per sequence], zero between launches
+    float *pieces;  // [workers * 2][heads per CTA][D + 1]
+    int grid;       // persistent CTAs
 };
+
+// Largest batch the balanced persistent decode schedule takes (its per-CTA tile prefix
+// over sequences lives in shared memory).
+constexpr int kStreamMaxBatch = 2048;
+// Persistent decode CTAs per SM and the SM count the workspace is sized for.
+constexpr int kStreamCtasPerSm = 2;
+constexpr int kStreamMaxSms = 160;
+constexpr int kStreamWorkersPerCta = 4;
+
+// Bytes at the start of a decode workspace that must be zero before a launch: the error
+// word header and, for the balanced schedule, one merge counter per (sequence, head).
+inline size_t decode_zero_prefix_bytes(int B, int Hq) {
+    return kWorkspaceHeader + ((size_t)B * Hq * sizeof(int) + 255) / 256 * 256;
+}
 
 // Launch the decode kernel (and nothing else) on `stream`.  The tensor maps describe the
 // K and V pools as 2-D arrays [num_pages*Hk*P rows][D].

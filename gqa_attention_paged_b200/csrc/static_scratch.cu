@@ -11,6 +11,7 @@
 
 #include <mutex>
 
+#include "gqa_internal.h"
 #include "gqa_paged.h"
 
 namespace {
@@ -58,9 +59,13 @@ extern "C" int gqa_paged_decode_static_scratch(
     void *ws = nullptr;
     const int st = scratch_address(&ws);
     if (st != GQA_OK) return st;
-    // The array keeps the previous call's contents; only the error word must start at
-    // zero (the split partials are fully rewritten by every call that uses them).
-    if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return GQA_ERR_LAUNCH;
+    // The array keeps the previous call's contents.  What must start at zero is cleared:
+    // the error word and the balanced schedule's merge counters (split partials and merge
+    // pieces are fully rewritten by every call that reads them).
+    size_t zero = sizeof(int);
+    if (B > 0 && Hq > 0) zero = gqa::decode_zero_prefix_bytes(B, Hq);
+    if (zero > (size_t)GQA_STATIC_SCRATCH_BYTES) zero = (size_t)GQA_STATIC_SCRATCH_BYTES;
+    if (cudaMemsetAsync(ws, 0, zero, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
     return gqa_paged_decode(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table,
                             pt_stride, seq_lens, B, Hq, Hk, head_dim, page_size, num_pages, scale,
                             num_splits, pack_gqa, out, lse, ws, (size_t)GQA_STATIC_SCRATCH_BYTES,

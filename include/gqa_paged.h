@@ -75,17 +75,21 @@ typedef enum {
 #define GQA_MAX_SPLITS 64
 
 /*
- * Bytes of workspace gqa_paged_decode() needs for `num_splits` splits (0 = the value
- * gqa_pick_splits() would choose for a context of up to max_seq_len tokens).  Layout:
- * a 256-byte header holding the device error word, then, when the call splits,
- * o_part fp32 [S][B*Hq][head_dim] and lse_part fp32 [S][B*Hq].
+ * Bytes of workspace gqa_paged_decode() needs for the same B, heads, head_dim, page_size,
+ * longest context (pt_stride * page_size), kv_dtype and num_splits.  Layout: a 256-byte
+ * header holding the device error word, then
+ *   num_splits = 0, B <= 2048 (balanced schedule): int32 merge counters [B*Hq] (rounded
+ *     up to 256 bytes) and the merge pieces, 2 per worker of the largest grid
+ *     (160 SMs x 3 CTAs x 4 workers), each min(Hq/Hk, 16) x (head_dim + 1) fp32;
+ *   split schedule with S > 1: o_part fp32 [S][B*Hq][head_dim] and lse_part fp32 [S][B*Hq].
  */
 size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int page_size,
                                        int max_seq_len, int kv_dtype, int num_splits);
 
 /*
- * Split count used when gqa_paged_decode() is called with num_splits = 0: a table
- * measured on B200 over batch size B, kv heads Hk and the longest context (tokens).
+ * Split count gqa_paged_decode() uses with num_splits = 0 when B is above the balanced
+ * schedule's limit (2048): chosen from B, kv heads Hk and the longest context (tokens)
+ * to give several waves of CTAs with at least 16 tiles of work each.
  */
 int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype);
 
@@ -105,16 +109,22 @@ int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype)
  *   seq_lens   int32 [B], each in [0, pt_stride * page_size]
  *   Hq % Hk == 0; head_dim in {64, 128}; page_size in {16, 32, 64}
  *   scale      softmax scale (commonly 1/sqrt(head_dim))
- *   num_splits 0 = automatic (gqa_pick_splits over max context pt_stride*page_size),
- *              else 1..GQA_MAX_SPLITS contiguous page-aligned ranges of
- *              ceil(np / num_splits) pages (np = ceil(seq_len / page_size)); the split
- *              results are merged with lse_combine on the same stream
+ *   num_splits 0 = automatic: for B <= 2048 a balanced persistent schedule: all
+ *              (sequence, kv head) tiles of 16 tokens are laid end to end and shared
+ *              equally by the workers of a fixed grid, and units cut between workers are
+ *              merged by log-sum-exp inside the same launch; for larger B, splits as
+ *              below with the count gqa_pick_splits gives for context pt_stride*page_size.
+ *              1..GQA_MAX_SPLITS: contiguous page-aligned ranges of ceil(np / num_splits)
+ *              pages (np = ceil(seq_len / page_size)), merged with lse_combine on the
+ *              same stream
  *   pack_gqa   1 (default): all heads of a group in one thread block, each KV page read
  *              once; 0: one query head per thread block (for comparison sweeps only)
  *   out        bf16 [B][Hq][head_dim]
  *   lse        fp32 [B][Hq] natural-log log-sum-exp, or NULL
  *   workspace  >= gqa_paged_decode_workspace_size(...) bytes, 256-byte aligned, zeroed
- *              before first use
+ *              before first use.  The balanced schedule keeps one merge counter per
+ *              (sequence, head) in it, back to zero at the end of every launch; after a
+ *              device-side error (see gqa_get_error) zero the workspace again.
  */
 int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                      const float *k_scale, const float *v_scale, int kv_dtype,

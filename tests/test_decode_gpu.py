@@ -88,7 +88,7 @@ def test_sweep_decode_batch(B):
         check(out[rows], lse[rows], ref_o, ref_l, what=f"sweep B={B} S={S}")
 
 
-@pytest.mark.parametrize("S", [1, 4])
+@pytest.mark.parametrize("S", [0, 1, 4])
 def test_sweep_decode_pack_off(S):
     case = inputs.sweep_decode(16, seed=3)
     ref_o, ref_l = oracle_decode(case)
@@ -123,7 +123,7 @@ def test_long70b_decode_fp8(S):
 def test_head_layouts_mha_mqa_and_odd_groups(Hq, Hk, D, P):
     case = inputs.make_decode_case(3, Hq, Hk, D, P, [1, 150, 333], seed=Hq * D + P)
     ref_o, ref_l = oracle_decode(case)
-    for S in (1, 3):
+    for S in (0, 1, 3):
         out, lse = run_decode(case, num_splits=S)
         check(out, lse, ref_o, ref_l, what=f"Hq={Hq} Hk={Hk} D={D} P={P} S={S}")
 
@@ -131,7 +131,7 @@ def test_head_layouts_mha_mqa_and_odd_groups(Hq, Hk, D, P):
 def test_empty_and_single_token_sequences():
     case = inputs.make_decode_case(5, 8, 2, 128, 16, [0, 1, 0, 16, 17], seed=21)
     ref_o, ref_l = oracle_decode(case)
-    for S in (1, 2, 5):
+    for S in (0, 1, 2, 5):
         out, lse = run_decode(case, num_splits=S)
         check(out, lse, ref_o, ref_l, what=f"empty S={S}")
         assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
@@ -197,9 +197,25 @@ def test_lse_combine_standalone():
     assert np.isneginf(lse[3]) and np.all(out[3] == 0)
 
 
-def test_repeated_calls_are_deterministic():
+@pytest.mark.parametrize("S", [0, 3])
+def test_repeated_calls_are_deterministic(S):
     case = inputs.llama7b_decode(seed=6, B=4)
     dev = to_dev(case)
-    a = run_decode(case, num_splits=3, dev=dev)
-    b = run_decode(case, num_splits=3, dev=dev)
+    ws = binding.new_workspace(binding.gqa_paged_decode_workspace_size(4, 32, 8, 128, 16, 2048, 0, S), DEV)
+    a = run_decode(case, num_splits=S, dev=dev, workspace=ws)
+    b = run_decode(case, num_splits=S, dev=dev, workspace=ws)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    if S == 0:  # merge counters are back to zero after every launch
+        hdr = 256
+        assert int(ws[hdr:hdr + 4 * 4 * 32].view(torch.int32).abs().sum()) == 0
+
+
+@pytest.mark.parametrize("lens", [[1], [2048], [16] * 37, [0, 0, 5], [3000, 1, 17, 0, 900, 4096]])
+def test_balanced_schedule_shapes(lens):
+    """The balanced persistent schedule (num_splits = 0) on batch shapes whose units are
+    cut between workers in many ways: one tile, one long sequence, many tiny ones, empty
+    sequences, a ragged mix."""
+    case = inputs.make_decode_case(len(lens), 32, 8, 128, 16, lens, seed=sum(lens) % 97)
+    ref_o, ref_l = oracle_decode(case)
+    out, lse = run_decode(case, num_splits=0)
+    check(out, lse, ref_o, ref_l, what=f"balanced {lens}")

@@ -1,0 +1,106 @@
+"""Host check of the balanced persistent decode schedule's integer arithmetic: the tile
+partition among workers, the owner of a tile, and the merge pieces of units that workers
+share.  The formulas are the ones decode_sk_kernel evaluates (restated here): worker W
+owns flat tiles [W*T//NW, (W+1)*T//NW); the owner of tile t is ((t+1)*NW + T-1)//T - 1;
+a unit cut between workers leaves one piece per worker, side 1 for the worker where the
+unit begins and side 0 for the others, and the last of them merges all pieces."""
+import itertools
+import random
+
+import pytest
+
+
+def start(W, T, NW):
+    return T if W >= NW else (W * T) // NW
+
+
+def owner(t, T, NW):
+    return ((t + 1) * NW + T - 1) // T - 1
+
+
+def schedule(tiles_per_seq, U, workers):
+    """Simulate every worker: returns (final writes, pieces) per unit, plus the slots."""
+    pre = [0]
+    for n in tiles_per_seq:
+        pre.append(pre[-1] + n)
+    T = U * pre[-1]
+    NW = min(workers, T)
+    finals, pieces, slots = {}, {}, {}
+    for W in range(workers):
+        s, e = start(W, T, NW), start(W + 1, T, NW)
+        for f in range(s, e):
+            b = next(bb for bb in range(len(tiles_per_seq)) if U * pre[bb + 1] > f)
+            nt = pre[b + 1] - pre[b]
+            local = f - U * pre[b]
+            y, tile = divmod(local, nt)
+            if tile != nt - 1 and f != e - 1:
+                continue
+            us = U * pre[b] + y * nt
+            ue = us + nt
+            if us >= s and ue <= e:
+                finals.setdefault((b, y), []).append(W)
+            else:
+                side = 0 if us < s else 1
+                key = (W, side)
+                assert key not in slots, "two units in one slot"
+                slots[key] = (b, y)
+                pieces.setdefault((b, y), []).append((W, side))
+    return T, NW, finals, pieces
+
+
+@pytest.mark.parametrize("workers", [1, 3, 4, 7, 16, 64])
+def test_partition_and_owner(workers):
+    for T in range(1, 300):
+        NW = min(workers, T)
+        cover = []
+        for W in range(workers):
+            cover += list(range(start(W, T, NW), start(W + 1, T, NW)))
+        assert cover == list(range(T))
+        sizes = [start(W + 1, T, NW) - start(W, T, NW) for W in range(NW)]
+        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+        for t in range(T):
+            W = owner(t, T, NW)
+            assert start(W, T, NW) <= t < start(W + 1, T, NW)
+
+
+def test_units_are_written_exactly_once():
+    rng = random.Random(0)
+    for trial in range(300):
+        B = rng.randint(1, 7)
+        tiles = [rng.choice([0, 1, 2, 3, 5, 8, 13, 40]) for _ in range(B)]
+        U = rng.choice([1, 2, 3, 8])
+        workers = rng.choice([1, 2, 4, 12, 32])
+        if sum(tiles) == 0:
+            continue
+        T, NW, finals, pieces = schedule(tiles, U, workers)
+        for b, n in enumerate(tiles):
+            for y in range(U):
+                key = (b, y)
+                if n == 0:
+                    assert key not in finals and key not in pieces
+                    continue
+                assert (key in finals) != (key in pieces)
+                if key in finals:
+                    assert len(finals[key]) == 1
+                    continue
+                us = U * sum(tiles[:b]) + y * n
+                ue = us + n
+                w0, w1 = owner(us, T, NW), owner(ue - 1, T, NW)
+                got = sorted(pieces[key])
+                want = sorted([(w0, 1)] + [(W, 0) for W in range(w0 + 1, w1 + 1)])
+                assert got == want, (tiles, U, workers, key)
+
+
+def test_slot_indices_stay_in_the_workspace():
+    """Slots W*2+side < 2 * (SMs * CTAs per SM * 4 workers), the bound the workspace is
+    sized for; counters b*U+y < B*Hq."""
+    sms, per_sm, wpc = 160, 3, 4
+    workers = sms * per_sm * wpc
+    for B, Hq, Hk, hpc in itertools.product([1, 5, 64], [8, 32, 64], [1, 8], [1, 4, 16]):
+        if Hq % Hk:
+            continue
+        g = Hq // Hk
+        hpc = min(hpc, g)
+        U = Hk * ((g + hpc - 1) // hpc)
+        assert B * U <= B * Hq
+        assert 2 * (workers - 1) + 1 < 2 * workers
