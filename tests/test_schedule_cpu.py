@@ -1,13 +1,18 @@
 """Host check of the balanced persistent decode schedule's integer arithmetic: the tile
 partition among workers, the owner of a tile, and the merge pieces of units that workers
 share.  The formulas are the ones decode_sk_kernel evaluates (restated here): worker W
-owns flat tiles [W*T//NW, (W+1)*T//NW); the owner of tile t is ((t+1)*NW + T-1)//T - 1;
+owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // 16)); the owner
+of tile t is ((t+1)*NW + T-1)//T - 1;
 a unit cut between workers leaves one piece per worker, side 1 for the worker where the
 unit begins and side 0 for the others, and the last of them merges all pieces."""
 import itertools
 import random
 
 import pytest
+
+
+def n_workers(workers, T):
+    return min(workers, max(1, T // 16))
 
 
 def start(W, T, NW):
@@ -24,7 +29,7 @@ def schedule(tiles_per_seq, U, workers):
     for n in tiles_per_seq:
         pre.append(pre[-1] + n)
     T = U * pre[-1]
-    NW = min(workers, T)
+    NW = n_workers(workers, T)
     finals, pieces, slots = {}, {}, {}
     for W in range(workers):
         s, e = start(W, T, NW), start(W + 1, T, NW)
@@ -51,13 +56,13 @@ def schedule(tiles_per_seq, U, workers):
 @pytest.mark.parametrize("workers", [1, 3, 4, 7, 16, 64])
 def test_partition_and_owner(workers):
     for T in range(1, 300):
-        NW = min(workers, T)
+        NW = n_workers(workers, T)
         cover = []
         for W in range(workers):
             cover += list(range(start(W, T, NW), start(W + 1, T, NW)))
         assert cover == list(range(T))
         sizes = [start(W + 1, T, NW) - start(W, T, NW) for W in range(NW)]
-        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= min(16, T)
         for t in range(T):
             W = owner(t, T, NW)
             assert start(W, T, NW) <= t < start(W + 1, T, NW)
@@ -67,7 +72,7 @@ def test_units_are_written_exactly_once():
     rng = random.Random(0)
     for trial in range(300):
         B = rng.randint(1, 7)
-        tiles = [rng.choice([0, 1, 2, 3, 5, 8, 13, 40]) for _ in range(B)]
+        tiles = [rng.choice([0, 1, 2, 3, 5, 8, 13, 40, 128]) for _ in range(B)]
         U = rng.choice([1, 2, 3, 8])
         workers = rng.choice([1, 2, 4, 12, 32])
         if sum(tiles) == 0:
@@ -94,7 +99,7 @@ def test_units_are_written_exactly_once():
 def test_slot_indices_stay_in_the_workspace():
     """Slots W*2+side < 2 * (SMs * CTAs per SM * 4 workers), the bound the workspace is
     sized for; counters b*U+y < B*Hq."""
-    sms, per_sm, wpc = 160, 3, 4
+    sms, per_sm, wpc = 160, 2, 4
     workers = sms * per_sm * wpc
     for B, Hq, Hk, hpc in itertools.product([1, 5, 64], [8, 32, 64], [1, 8], [1, 4, 16]):
         if Hq % Hk:
