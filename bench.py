@@ -200,8 +200,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", action="store_true",
-                    help="print one line per (B, splits, pack) point instead of the headline")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+                    help="decode: the headline (paged GQA decode); prefill: causal chunked "
+                         "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]")
     return ap.parse_args()
 
 
@@ -210,12 +211,86 @@ def workload_name(a):
             f"kv={a.kv}")
 
 
+def prefill_flops(prior_lens, q_lens, Hq, D):
+    """4*Hq*D per unmasked (query, key) pair: row i of a chunk of Lq after `prior` keys
+    sees prior + i + 1 keys."""
+    pairs = sum(int(Lq) * int(p) + int(Lq) * (int(Lq) + 1) // 2 for p, Lq in zip(prior_lens, q_lens))
+    return 4 * Hq * D * pairs
+
+
+def tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def run_prefill_bench(a):
+    import torch
+    from gqa_attention_paged_b200 import binding, inputs
+
+    dev = torch.device("cuda", 0)
+    case = inputs.chunked_prefill(seed=a.seed)
+    kv = case.kv
+    q, cu = case.q.to(dev), case.cu_q.to(dev)
+    kp, vp, pt, sl = kv.k_pages.to(dev), kv.v_pages.to(dev), kv.page_table.to(dev), kv.seq_lens.to(dev)
+    T, Hq, D = case.q.shape
+    out = torch.empty(T, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    ws = binding.new_workspace(binding.gqa_paged_prefill_workspace_size(T, Hq, D), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.gqa_paged_prefill(q, cu, kp, vp, pt, sl, case.scale, case.max_q_len, out=out,
+                                  lse=lse, workspace=ws, stream=stream)
+
+    step()
+    torch.cuda.synchronize(dev)
+    assert binding.gqa_get_error(ws) == 0 and torch.isfinite(out.float()).all()
+    for _ in range(max(3, a.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / a.steps
+    clk = clocks.stop()
+    q_lens = (case.cu_q[1:] - case.cu_q[:-1]).tolist()
+    prior = [int(L) - int(x) for L, x in zip(kv.seq_lens.tolist(), q_lens)]
+    flops = prefill_flops(prior, q_lens, Hq, D)
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, kind = tensor_peak()
+    print(json.dumps({
+        "metric": "causal chunked prefill over a paged KV cache: TFLOP/s (unmasked pairs)",
+        "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps,
+        "warmup": max(3, a.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v)",
+        "config": {"workload": "chunked prefill B=8 Lq=512 prior~U[0,4096] Hq=32 Hk=8 D=128 P=16",
+                   "flops_per_step": flops, "prior_lens": prior},
+        "tokens_per_s": round(sum(q_lens) / (ms * 1e-3), 1),
+        "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tf / peak, 4), "traffic": None,
+                     "peak_source": f"{kind} (bf16_tflops, burst cuBLAS GEMM)"},
+        "gpu_launches": a.steps, "clocks": clk}))
+    return 0
+
+
 def main():
     a = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if a.workload == "prefill" and a.impl == "ours":
+        return run_prefill_bench(a)
     if a.impl == "reference":
         if rank != 0:
             return 0

@@ -5,25 +5,28 @@
 // prefill); its K/V are already the last Lq cached tokens, and query row i (position
 // L - Lq + i) attends to keys 0 .. L - Lq + i.
 //
-// One CTA = (query tile, kv head, sequence).  The tile packs the g query heads of the
+// One CTA = (two query tiles, kv head, sequence).  A tile packs the g query heads of the
 // group with T = 128 / g tokens into 128 rows, row r = (token r / g, head r % g)
 // (PackGQA: "解锁GQA性能潜力：从批量大小敏感性到高效优化实践", PackGQA / NumSplits
-// section), so each K/V tile feeds every head of the group.  The attention itself is the
-// tiled fused form ("TensorRT-LLM与TensorRT核心差异解析", section 4.2.1): per tile of 128
-// keys, S = Q K^T on tcgen05 into tensor memory, an fp32 online softmax in registers,
-// P (bf16) into shared memory, and O += P V on tcgen05 into tensor memory.
+// section), so each K/V tile feeds every head of the group, twice (once per query tile).
+// The attention is the tiled fused form ("TensorRT-LLM与TensorRT核心差异解析", section
+// 4.2.1): per 128-key tile, S = Q K^T on tcgen05 into tensor memory, an fp32 online
+// softmax in registers, P written back into tensor memory over S, and O += P V on
+// tcgen05 with P read from tensor memory.
 //
-// Warp roles (192 threads):
-//   warp 0   TMA producer: Q tile (3-D map over [total_q][Hq][D]), then K/V tiles, 16
-//            keys per copy, gathered page by page through the page table (2-stage ring).
-//   warp 1   allocates tensor memory (S: 128 columns, O: 128 columns) and issues the MMAs
-//            (one thread), S_{j+1} overlapping the softmax of tile j.
-//   warps 2-5 softmax / correction / epilogue: thread = one row (tensor-memory lane).
-// P is written as a bf16 value plus its bf16 residual and O += P_hi V + P_lo V, so the
-// probabilities keep ~16 significant bits (a single bf16 P loses up to 2^-9 of each
-// weight, visible as ~5e-3 errors in short rows whose terms cancel).
-// The running max is only moved when a row's max grows by more than 2^8, so O (kept in
-// tensor memory) is rescaled rarely; the final O / l is exact for any reference max.
+// Warp roles (320 threads):
+//   warp 0     TMA producer: both Q tiles (3-D map over [total_q][Hq][D]), then K and V
+//              tiles, 16 keys per copy, gathered page by page through the page table.
+//   warp 1     allocates all 512 tensor-memory columns (S0, S1, O0, O1) and issues the
+//              MMAs from one thread in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so the
+//              tensor core works on one query tile while the other one's softmax runs.
+//   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1; a thread owns one row
+//              (one tensor-memory lane).
+// P is stored as a bf16 value plus its bf16 residual and O += P_hi V + P_lo V, which
+// keeps the probabilities at ~16 significant bits (a single bf16 P loses up to 2^-9 of
+// each weight, visible as ~5e-3 errors in short rows whose terms cancel).
+// The running max is only moved when a row's max grows by more than 2^8, so O is
+// rescaled rarely; the final O / l is exact for any reference max.
 // Every wait is bounded; on expiry the kernel records GQA_ERR_TIMEOUT, finishes its
 // outstanding copies and MMAs (bounded), frees its tensor memory and returns.
 #include "gqa_device.cuh"
@@ -32,11 +35,12 @@
 namespace gqa {
 namespace {
 
-constexpr int kM = 128;                // packed query rows per tile
+constexpr int kM = 128;                // packed query rows per query tile
+constexpr int kQT = 2;                 // query tiles per CTA
 constexpr int kN = 128;                // keys per KV tile
 constexpr int kD = 128;                // head dim
 constexpr int kStages = 2;             // K/V ring depth
-constexpr int kThreadsP = 192;
+constexpr int kThreadsP = 320;
 constexpr int kHalfBytes = kM * 128;   // one 64-column (128-byte) half of a 128-row tile
 constexpr int kTileBytesP = 2 * kHalfBytes;
 constexpr int kChunk = 16;             // keys per TMA copy (one box)
@@ -47,17 +51,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned kAll = 0xffffffffu;
 
 struct alignas(1024) PSmem {
-    uint8_t q[kTileBytesP];
+    uint8_t q[kQT][kTileBytesP];
     uint8_t k[kStages][kTileBytesP];
     uint8_t v[kStages][kTileBytesP];
-    uint8_t p[kTileBytesP];     // bf16 part of P
-    uint8_t p_lo[kTileBytesP];  // bf16 residual of P (P - p): two MMAs keep P at ~16 bits
     uint64_t q_full;
-    uint64_t kv_full[kStages];
-    uint64_t kv_empty[kStages];
-    uint64_t s_full, s_free, p_full, pv_done, mma_done;
+    uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    uint64_t s_full[kQT], p_full[kQT], pv_done[kQT];
+    uint64_t mma_done;
     uint32_t tmem_base;
-    int abort_flag;
 };
 
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity) {
@@ -73,49 +74,55 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                                            ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z, kvh = blockIdx.y;
-    const int qt = gridDim.x - 1 - blockIdx.x;  // longest (latest) tiles first
+    const int ct = gridDim.x - 1 - blockIdx.x;  // longest (latest) tiles first
     const int g = a.Hq / a.Hk;
     const int q0 = a.cu_q[b];
     const int Lq = a.cu_q[b + 1] - q0;
-    const int i0 = qt * T;
-    if (blockIdx.x == 0 && threadIdx.x == 0 && Lq > (int)gridDim.x * T)
+    const int i0 = ct * kQT * T;  // first token of query tile 0
+    if (blockIdx.x == 0 && threadIdx.x == 0 && Lq > (int)gridDim.x * kQT * T)
         set_error(a.err, GQA_ERR_SHAPE);  // max_q_len below a chunk length
     if (i0 >= Lq) return;  // uniform for the whole CTA
-    int L = a.seq_lens[b];
+    const int L = a.seq_lens[b];
     const int P = a.P;
     if (L < Lq || L > a.pt_stride * P) {
         if (threadIdx.x == 0) set_error(a.err, GQA_ERR_BAD_PAGE);
         return;
     }
-    const int ntok = min(T, Lq - i0);
-    const int rows_valid = ntok * g;
-    const int pos_hi = L - Lq + i0 + ntok - 1;
-    const int n_kv = a.causal ? pos_hi / kN + 1 : (L + kN - 1) / kN;
+    // KV tiles each query tile needs (0 when the tile has no token of the chunk)
+    int n_kv_q[kQT];
+#pragma unroll
+    for (int q = 0; q < kQT; ++q) {
+        const int ntok = min(T, Lq - (i0 + q * T));
+        n_kv_q[q] = ntok <= 0 ? 0
+                    : a.causal ? (L - Lq + i0 + q * T + ntok - 1) / kN + 1
+                               : (L + kN - 1) / kN;
+    }
+    const int n_kv = max(n_kv_q[0], n_kv_q[1]);
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
-        mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.s_free, 4);
-        mbar_init(&sm.p_full, 4);
-        mbar_init(&sm.pv_done, 1);
+        for (int q = 0; q < kQT; ++q) {
+            mbar_init(&sm.s_full[q], 1);
+            mbar_init(&sm.p_full[q], 4);
+            mbar_init(&sm.pv_done[q], 1);
+        }
         mbar_init(&sm.mma_done, 1);
-        sm.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, 256);
+        tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tS = tmem, tO = tmem + 128;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -124,10 +131,11 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             prefetch_tensormap(&qmap);
             prefetch_tensormap(&kmap);
             prefetch_tensormap(&vmap);
-            mbar_arrive_expect_tx(&sm.q_full, 2 * g * T * 128);
-            tma_load_3d(sm.q, &qmap, &sm.q_full, 0, kvh * g, q0 + i0, policy_evict_first());
-            tma_load_3d(sm.q + kHalfBytes, &qmap, &sm.q_full, 64, kvh * g, q0 + i0,
-                        policy_evict_first());
+            mbar_arrive_expect_tx(&sm.q_full, kQT * 2 * g * T * 128);
+            for (int q = 0; q < kQT; ++q)
+                for (int h = 0; h < 2; ++h)
+                    tma_load_3d(sm.q[q] + h * kHalfBytes, &qmap, &sm.q_full, 64 * h, kvh * g,
+                                q0 + i0 + q * T, policy_evict_first());
         }
         const int32_t *pt = a.page_table + (size_t)b * a.pt_stride;
         int issued = 0;
@@ -152,28 +160,34 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     set_error(a.err, GQA_ERR_TIMEOUT);
                     fail = true;
                 } else {
-                    mbar_arrive_expect_tx(&sm.kv_full[stage], __popc(mask) * 4 * kChunkBytes);
+                    // K first: the S MMAs can start before V lands
+                    mbar_arrive_expect_tx(&sm.k_full[stage], __popc(mask) * 2 * kChunkBytes);
 #pragma unroll
-                    for (int c = 0; c < kN / kChunk; ++c) {
-                        if (!((mask >> c) & 1u)) continue;
+                    for (int c = 0; c < kN / kChunk; ++c)
+                        if ((mask >> c) & 1u)
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            tma_load_2d(sm.k[stage] + h * kHalfBytes + c * kChunkBytes, &kmap,
-                                        &sm.kv_full[stage], 64 * h, rows[c], pol_kv);
-                            tma_load_2d(sm.v[stage] + h * kHalfBytes + c * kChunkBytes, &vmap,
-                                        &sm.kv_full[stage], 64 * h, rows[c], pol_kv);
-                        }
-                    }
+                            for (int h = 0; h < 2; ++h)
+                                tma_load_2d(sm.k[stage] + h * kHalfBytes + c * kChunkBytes, &kmap,
+                                            &sm.k_full[stage], 64 * h, rows[c], pol_kv);
+                    mbar_arrive_expect_tx(&sm.v_full[stage], __popc(mask) * 2 * kChunkBytes);
+#pragma unroll
+                    for (int c = 0; c < kN / kChunk; ++c)
+                        if ((mask >> c) & 1u)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                tma_load_2d(sm.v[stage] + h * kHalfBytes + c * kChunkBytes, &vmap,
+                                            &sm.v_full[stage], 64 * h, rows[c], pol_kv);
                     issued = j + 1;
                 }
             }
             fail = __shfl_sync(kAll, fail, 0);
         }
         if (lane == 0) {
-            // no copy may outlive the CTA: wait for the Q tile and the last issued tiles
+            // no copy may outlive the CTA: wait for the Q tiles and the last issued K/V tiles
             if (!mbar_wait(&sm.q_full, 0)) set_error(a.err, GQA_ERR_TIMEOUT);
             for (int j = max(0, issued - kStages); j < issued; ++j)
-                if (!mbar_wait(&sm.kv_full[j % kStages], (j / kStages) & 1)) {
+                if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1) ||
+                    !mbar_wait(&sm.v_full[j % kStages], (j / kStages) & 1)) {
                     set_error(a.err, GQA_ERR_TIMEOUT);
                     break;
                 }
@@ -181,51 +195,64 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);   // Q, K both K-major
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, kD, 0, 1);   // P K-major, V MN-major
-        const uint32_t qa = smem_u32(sm.q), pa = smem_u32(sm.p), pla = smem_u32(sm.p_lo);
-        bool ok = wait_all(&sm.q_full, 0) && wait_all(&sm.kv_full[0], 0);
-        int committed_pv = 0;  // PV MMAs committed to pv_done
-        if (ok) {
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, kD, 0, 1);   // P (TMEM), V MN-major
+        bool ok = wait_all(&sm.q_full, 0);
+        // S_q(j) = Q_q K_j^T into tensor-memory columns [128 q, 128 q + 128)
+        auto issue_s = [&](int q, int j) -> bool {
+            const int stage = j % kStages;
+            if (!wait_all(&sm.k_full[stage], (j / kStages) & 1)) return false;
             tc_fence_after_sync();
             if (lane == 0) {
-                const uint32_t ka = smem_u32(sm.k[0]);
+                const uint32_t qa = smem_u32(sm.q[q]), ka = smem_u32(sm.k[stage]);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    tc_mma_ss(tS, smem_desc_sw128(qa + off, 16, 1024),
+                    tc_mma_ss(tmem + 128 * q, smem_desc_sw128(qa + off, 16, 1024),
                               smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
                 }
-                tc_commit(&sm.s_full);
+                tc_commit(&sm.s_full[q]);
             }
             __syncwarp();
-        }
+            return true;
+        };
+        // O_q += P_q(j) V_j with P_q(j) in S_q's columns: keys 32c..32c+31 as bf16 value
+        // pairs in columns [32c, 32c+16) and residual pairs in [32c+16, 32c+32)
+        auto issue_pv = [&](int q, int j) -> bool {
+            const int stage = j % kStages;
+            if (!wait_all(&sm.p_full[q], j & 1) ||
+                !wait_all(&sm.v_full[stage], (j / kStages) & 1))
+                return false;
+            tc_fence_after_sync();
+            if (lane == 0) {
+                const uint32_t va = smem_u32(sm.v[stage]);
+                const uint32_t tp = tmem + 128 * q, to = tmem + 256 + 128 * q;
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk)
+                    tc_mma_ts(to, tp + 32 * (kk >> 1) + 8 * (kk & 1),
+                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                              (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk)
+                    tc_mma_ts(to, tp + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
+                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
+                tc_commit(&sm.pv_done[q]);
+            }
+            __syncwarp();
+            return true;
+        };
+        for (int q = 0; q < kQT && ok; ++q)
+            if (n_kv_q[q] > 0) ok = issue_s(q, 0);
         for (int j = 0; j < n_kv && ok; ++j) {
             const int stage = j % kStages;
-            if (j + 1 < n_kv) {
-                ok = wait_all(&sm.kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1) &&
-                     wait_all(&sm.s_free, j & 1);
-                if (!ok) break;
-                tc_fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t ka = smem_u32(sm.k[(j + 1) % kStages]);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                        tc_mma_ss(tS, smem_desc_sw128(qa + off, 16, 1024),
-                                  smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
-                    }
-                    tc_commit(&sm.s_full);
-                }
-                __syncwarp();
-            }
-            ok = wait_all(&sm.p_full, j & 1);
-            if (!ok) break;
-            tc_fence_after_sync();
             if (j == n_kv - 1) {
                 // keys at or past L hold anything (even NaN): zero those V rows so their
                 // zero weights contribute exactly zero.
                 const int valid = L - j * kN;
                 if (valid < kN) {
+                    if (!wait_all(&sm.v_full[stage], (j / kStages) & 1)) {
+                        ok = false;
+                        break;
+                    }
                     for (int e = lane; e < (kN - valid) * 16; e += 32) {
                         const int r = valid + (e >> 4), c16 = e & 15;
                         *reinterpret_cast<uint4 *>(sm.v[stage] + (c16 >> 3) * kHalfBytes + r * 128 +
@@ -235,133 +262,118 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     __syncwarp();
                 }
             }
-            if (lane == 0) {
-                const uint32_t va = smem_u32(sm.v[stage]);
-#pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    tc_mma_ss(tO, smem_desc_sw128(pa + aoff, 16, 1024),
-                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                              (j > 0 || kk > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    tc_mma_ss(tO, smem_desc_sw128(pla + aoff, 16, 1024),
-                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
-                }
-                tc_commit(&sm.pv_done);
-                tc_commit(&sm.kv_empty[stage]);
+            for (int q = 0; q < kQT && ok; ++q) {
+                if (j >= n_kv_q[q]) continue;
+                ok = issue_pv(q, j);
+                if (ok && j + 1 < n_kv_q[q]) ok = issue_s(q, j + 1);
             }
-            committed_pv = j + 1;
+            if (ok && lane == 0) tc_commit(&sm.kv_empty[stage]);
             __syncwarp();
         }
         if (!ok && lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
-        (void)committed_pv;
         // every MMA issued must be finished before tensor memory is released
         if (lane == 0) tc_commit(&sm.mma_done);
         __syncwarp();
         if (!wait_all(&sm.mma_done, 0) && lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
     } else {
-        // ------------------------------------------------------------ softmax warps
-        const int quad = warp & 3;
+        // ------------------------------------------------------------ softmax warpgroups
+        const int q = (warp - 2) / 4;  // query tile
+        const int quad = warp & 3;     // tensor-memory lane quadrant this warp may access
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const bool valid_row = row < rows_valid;
-        const int tok = i0 + row / g;
+        const uint32_t tS = tmem + 128 * q + lane_off, tO = tmem + 256 + 128 * q + lane_off;
+        const int nk = n_kv_q[q];
+        const int ntok = min(T, Lq - (i0 + q * T));
+        const bool valid_row = row < ntok * g;
+        const int tok = i0 + q * T + row / g;
         const int hh = row % g;
         const int lim = a.causal ? min(L - Lq + tok, L - 1) : L - 1;  // last visible key
-        const float scale_log2 = a.scale * kLog2eP;
+        const float c = a.scale * kLog2eP;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            if (!wait_all(&sm.s_full, j & 1)) {
+        for (int j = 0; j < nk; ++j) {
+            if (!wait_all(&sm.s_full[q], j & 1)) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + 32 * c, sr[c]);
-            tmem_wait_ld();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_free);
-
+            // Pass 1: row max over the visible keys of this tile (S stays in tensor memory;
+            // reading it twice keeps the row's 128 scores out of the register file).
             const int nvis = lim - j * kN + 1;  // keys of this tile the row may see
             float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int cc = 0; cc < 4; cc += 2) {
+                uint32_t sa[32], sb[32];
+                tmem_ld32(tS + 32 * cc, sa);
+                tmem_ld32(tS + 32 * cc + 32, sb);
+                tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float x = (32 * c + e < nvis) ? __uint_as_float(sr[c][e]) * scale_log2
-                                                        : -INFINITY;
-                    sr[c][e] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                    mx = fmaxf(mx, (32 * cc + e < nvis) ? __uint_as_float(sa[e]) : -INFINITY);
+                    mx = fmaxf(mx, (32 * cc + 32 + e < nvis) ? __uint_as_float(sb[e]) : -INFINITY);
                 }
+            }
+            mx *= c;  // c > 0: the max commutes with the scale
             const bool need = mx > m_ref + kRescaleThreshold;
             const float new_ref = need ? mx : m_ref;
             const float mref0 = new_ref == -INFINITY ? 0.f : new_ref;
-            const float alpha = fast_exp2(m_ref - mref0);
+            const float alpha = ex2_approx(m_ref - mref0);
 
-            if (j > 0) {
-                if (!wait_all(&sm.pv_done, (j - 1) & 1)) {
+            if (j > 0 && __any_sync(kAll, need)) {
+                // O must not be touched while PV(j-1) still accumulates into it
+                if (!wait_all(&sm.pv_done[q], (j - 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                if (__any_sync(kAll, need)) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + lane_off + 32 * c, o);
-                        tmem_wait_ld();
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * cc, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tO + lane_off + 32 * c, o);
-                    }
-                    tmem_wait_st();
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tO + 32 * cc, o);
                 }
             }
-            // P row (bf16 value + bf16 residual) into the swizzled K-major tiles: 16 chunks
-            // of 8 keys each.
+            // Pass 2: P = 2^(s*c - ref) (0 past the visible keys), written over S in
+            // tensor memory chunk by chunk: the 32 keys of chunk cc (columns [32cc, 32cc+32)
+            // of S) become 16 columns of bf16 value pairs then 16 of bf16 residual pairs in
+            // those same columns, so a store never lands on scores not yet read.
             float sum = 0.f;
-            uint8_t *prow = sm.p + row * 128;
-            uint8_t *plrow = sm.p_lo + row * 128;
 #pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
-                float pv[8];
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t sr[32];
+                tmem_ld32(tS + 32 * cc, sr);
+                tmem_wait_ld();
+                uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    pv[e] = fast_exp2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + e]) - mref0);
-                    sum += pv[e];
+                for (int e = 0; e < 16; ++e) {
+                    const int k0 = 32 * cc + 2 * e;
+                    const float p0 = k0 < nvis ? ex2_approx(__uint_as_float(sr[2 * e]) * c - mref0) : 0.f;
+                    const float p1 = k0 + 1 < nvis ? ex2_approx(__uint_as_float(sr[2 * e + 1]) * c - mref0) : 0.f;
+                    sum += p0 + p1;
+                    split_bf16x2(p0, p1, hi[e], lo[e]);
                 }
-                uint4 w, wl;
-                split_bf16x2(pv[0], pv[1], w.x, wl.x);
-                split_bf16x2(pv[2], pv[3], w.y, wl.y);
-                split_bf16x2(pv[4], pv[5], w.z, wl.z);
-                split_bf16x2(pv[6], pv[7], w.w, wl.w);
-                const int off = (ch >> 3) * kHalfBytes + (((ch & 7) ^ (row & 7)) << 4);
-                *reinterpret_cast<uint4 *>(prow + off) = w;
-                *reinterpret_cast<uint4 *>(plrow + off) = wl;
+                tmem_st16(tS + 32 * cc, hi);
+                tmem_st16(tS + 32 * cc + 16, lo);
             }
+            tmem_wait_st();
             l = l * alpha + sum;
             m_ref = new_ref;
-            fence_proxy_async_smem();
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full);
+            if (lane == 0) mbar_arrive(&sm.p_full[q]);
         }
-        if (ok && wait_all(&sm.pv_done, (n_kv - 1) & 1)) {
+        if (nk > 0 && ok && wait_all(&sm.pv_done[q], (nk - 1) & 1)) {
             tc_fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) +
                                  ((size_t)(q0 + tok) * a.Hq + kvh * g + hh) * kD;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int cc = 0; cc < 4; ++cc) {
                 uint32_t o[32];
-                tmem_ld32(tO + lane_off + 32 * c, o);
+                tmem_ld32(tO + 32 * cc, o);
                 tmem_wait_ld();
                 if (valid_row) {
 #pragma unroll
@@ -371,14 +383,14 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                         w.y = pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
                         w.z = pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
                         w.w = pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(dst + 32 * c + e) = w;
+                        *reinterpret_cast<uint4 *>(dst + 32 * cc + e) = w;
                     }
                 }
             }
             if (valid_row && a.lse)
                 a.lse[(size_t)(q0 + tok) * a.Hq + kvh * g + hh] =
                     l > 0.f ? (m_ref + __log2f(l)) * kLn2P : -INFINITY;
-        } else if (lane == 0) {
+        } else if (nk > 0 && lane == 0) {
             set_error(a.err, GQA_ERR_TIMEOUT);
         }
     }
@@ -387,7 +399,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -401,7 +413,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap, const 
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int tiles = (a.max_q_len + T - 1) / T;
+    const int tiles = (a.max_q_len + kQT * T - 1) / (kQT * T);
     if (tiles == 0 || a.B == 0) return cudaSuccess;
     dim3 grid(tiles, a.Hk, a.B);
     prefill_kernel<<<grid, kThreadsP, smem, stream>>>(kmap, vmap, qmap, a, T);
