@@ -244,7 +244,7 @@ int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
         return GQA_ERR_NULL;
     if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || Hk > 65535 ||
         Hq / Hk > 128 || head_dim != 128 || !valid_page_size(page_size) || num_pages <= 0 ||
-        pt_stride <= 0 || total_q < 0 || max_q_len < 0 ||
+        pt_stride <= 0 || total_q < 0 || max_q_len < 0 || !(scale > 0.f) ||
         (int64_t)num_pages * Hk * page_size > INT32_MAX ||
         (int64_t)pt_stride * page_size > INT32_MAX)
         return GQA_ERR_SHAPE;

@@ -300,19 +300,25 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             // Pass 1: row max over the visible keys of this tile (S stays in tensor memory;
             // reading it twice keeps the row's 128 scores out of the register file).
             const int nvis = lim - j * kN + 1;  // keys of this tile the row may see
-            float mx = -INFINITY;
+            float mx = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-            for (int cc = 0; cc < 4; cc += 2) {
-                uint32_t sa[32], sb[32];
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t sa[32];
                 tmem_ld32(tS + 32 * cc, sa);
-                tmem_ld32(tS + 32 * cc + 32, sb);
                 tmem_wait_ld();
+                if (nvis >= 32 * cc + 32) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    mx = fmaxf(mx, (32 * cc + e < nvis) ? __uint_as_float(sa[e]) : -INFINITY);
-                    mx = fmaxf(mx, (32 * cc + 32 + e < nvis) ? __uint_as_float(sb[e]) : -INFINITY);
+                    for (int e = 0; e < 32; e += 2) {
+                        mx = fmaxf(mx, __uint_as_float(sa[e]));
+                        mx1 = fmaxf(mx1, __uint_as_float(sa[e + 1]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        mx = fmaxf(mx, (32 * cc + e < nvis) ? __uint_as_float(sa[e]) : -INFINITY);
                 }
             }
+            mx = fmaxf(mx, mx1);
             mx *= c;  // c > 0: the max commutes with the scale
             const bool need = mx > m_ref + kRescaleThreshold;
             const float new_ref = need ? mx : m_ref;
@@ -339,25 +345,45 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             // Pass 2: P = 2^(s*c - ref) (0 past the visible keys), written over S in
             // tensor memory chunk by chunk: the 32 keys of chunk cc (columns [32cc, 32cc+32)
             // of S) become 16 columns of bf16 value pairs then 16 of bf16 residual pairs in
-            // those same columns, so a store never lands on scores not yet read.
-            float sum = 0.f;
+            // those same columns, so a store never lands on scores not yet read.  Keys go
+            // in pairs through the paired fp32 instructions.
+            const unsigned long long c2 = f2_pack(c, c), nref2 = f2_pack(-mref0, -mref0);
+            const unsigned long long neg1 = f2_pack(-1.f, -1.f);
+            unsigned long long sum2 = 0ull;  // (0.f, 0.f)
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t sr[32];
                 tmem_ld32(tS + 32 * cc, sr);
                 tmem_wait_ld();
+                if (nvis < 32 * cc + 32) {  // diagonal / tail tile: scores past nvis -> -inf
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * cc + e >= nvis) sr[e] = __float_as_uint(-INFINITY);
+                }
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int k0 = 32 * cc + 2 * e;
-                    const float p0 = k0 < nvis ? ex2_approx(__uint_as_float(sr[2 * e]) * c - mref0) : 0.f;
-                    const float p1 = k0 + 1 < nvis ? ex2_approx(__uint_as_float(sr[2 * e + 1]) * c - mref0) : 0.f;
-                    sum += p0 + p1;
-                    split_bf16x2(p0, p1, hi[e], lo[e]);
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                     c2, nref2), x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    const unsigned long long pp = f2_pack(p0, p1);
+                    sum2 = f2_add(sum2, pp);
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    hi[e] = *reinterpret_cast<uint32_t *>(&h);
+                    // residual: p - float(bf16(p)), exact in fp32
+                    const unsigned long long hf = f2_pack(__uint_as_float(hi[e] << 16),
+                                                          __uint_as_float(hi[e] & 0xffff0000u));
+                    float r0, r1;
+                    f2_unpack(f2_fma(hf, neg1, pp), r0, r1);
+                    lo[e] = pack_bf16(r0, r1);
                 }
                 tmem_st16(tS + 32 * cc, hi);
                 tmem_st16(tS + 32 * cc + 16, lo);
             }
+            float sum, sum_hi;
+            f2_unpack(sum2, sum, sum_hi);
+            sum += sum_hi;
             tmem_wait_st();
             l = l * alpha + sum;
             m_ref = new_ref;

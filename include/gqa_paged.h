@@ -194,7 +194,7 @@ size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim);
  *   cu_q       int32 [B+1], cu_q[0] = 0, nondecreasing, cu_q[B] = total_q,
  *              cu_q[b+1] - cu_q[b] <= max_q_len and <= seq_lens[b]
  *   k_pages, v_pages, page_table, pt_stride, seq_lens: as for decode (bf16 KV only)
- *   head_dim   128; page_size in {16, 32, 64}
+ *   head_dim   128; page_size in {16, 32, 64}; Hq / Hk <= 128; scale > 0
  *   out        bf16 [total_q][Hq][head_dim];  lse fp32 [total_q][Hq] or NULL
  *   workspace  >= gqa_paged_prefill_workspace_size(...) bytes, zeroed before first use
  */

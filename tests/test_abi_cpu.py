@@ -100,3 +100,20 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         binding.gqa_paged_decode(q, kp, kp, torch.zeros(1, 4, dtype=torch.int32),
                                  torch.ones(1, dtype=torch.int32), 0.125)
+
+
+def test_prefill_rejects_bad_arguments_on_the_host():
+    lib = binding.load()
+    def call(**kw):
+        args = dict(q=_fake(), cu=_fake(), k=_fake(), v=_fake(), pt=_fake(), pts=8, sl=_fake(),
+                    B=2, Hq=8, Hk=2, D=128, P=16, npg=16, scale=0.1, causal=1, tq=10, mq=5,
+                    out=_fake(), lse=None, ws=_fake(), wsb=256, st=None)
+        args.update(kw)
+        return lib.gqa_paged_prefill(*args.values())
+    assert call(q=None) == -1
+    assert call(D=64) == -2
+    assert call(scale=0.0) == -2
+    assert call(scale=-1.0) == -2
+    assert call(Hq=6, Hk=4) == -2
+    assert call(wsb=16) == -5
+    assert call(q=_fake(0x10008)) == -9
