@@ -200,13 +200,16 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "long70b"],
                     help="decode: the headline (paged GQA decode); prefill: causal chunked "
-                         "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]")
+                         "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]; "
+                         "long70b: B=4 decode at 8K/16K/24K/32K, Hq=64 Hk=8, page 64 (--kv)")
     return ap.parse_args()
 
 
 def workload_name(a):
+    if a.workload == "long70b":
+        return f"paged GQA decode, 70B-shaped long context: B=4 ctx={{8K,16K,24K,32K}} Hq=64 Hk=8 D=128 page_size=64 kv={a.kv}"
     return (f"paged GQA decode, B={a.B} ctx={a.ctx} Hq=32 Hk=8 D=128 page_size=16 "
             f"kv={a.kv}")
 
@@ -311,7 +314,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    case = inputs.sweep_decode(a.B, seed=rank_seed(a.seed, rank), ctx=a.ctx, kv_dtype=a.kv)
+    if a.workload == "long70b":
+        case = inputs.long70b_decode(seed=rank_seed(a.seed, rank), kv_dtype=a.kv)
+        a.B, a.ctx = 4, 32768
+    else:
+        case = inputs.sweep_decode(a.B, seed=rank_seed(a.seed, rank), ctx=a.ctx, kv_dtype=a.kv)
     kv = case.kv
     q = case.q.to(dev)
     kp, vp = kv.k_pages.to(dev), kv.v_pages.to(dev)
@@ -319,7 +326,7 @@ def main():
     vs = None if kv.v_scale is None else kv.v_scale.to(dev)
     pt, sl = kv.page_table.to(dev), kv.seq_lens.to(dev)
     elem = 1 if a.kv == "fp8_e4m3" else 2
-    B, Hq, Hk, D, P = a.B, 32, 8, 128, 16
+    B, Hq, Hk, D, P = a.B, case.Hq, case.Hk, case.head_dim, kv.page_size
     kvc = binding.GQA_KV_FP8_E4M3 if elem == 1 else binding.GQA_KV_BF16
     balanced = a.splits == 0 and B <= 2048  # num_splits = 0: the balanced persistent schedule
     S = a.splits if a.splits > 0 else (0 if balanced else

@@ -38,14 +38,15 @@ bool aligned(const void *p, size_t n) { return (reinterpret_cast<uintptr_t>(p) %
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// 2-D view [rows][D] of a KV pool, box = (128 bytes of a row) x 16 rows, 128B swizzle.
-int encode_kv_map(CUtensorMap *map, const void *pages, int kv_dtype, int D, int64_t rows) {
+// 2-D view [rows][D] of a KV pool, box = (128 bytes of a row) x box_rows rows, 128B swizzle.
+int encode_kv_map(CUtensorMap *map, const void *pages, int kv_dtype, int D, int64_t rows,
+                  int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return GQA_ERR_LAUNCH;
     const int elt = kv_dtype == GQA_KV_FP8_E4M3 ? 1 : 2;
     cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     cuuint64_t gstride[1] = {(cuuint64_t)D * elt};
-    cuuint32_t box[2] = {(cuuint32_t)(128 / elt), (cuuint32_t)kDecodeTileTokens};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / elt), (cuuint32_t)box_rows};
     cuuint32_t estride[2] = {1, 1};
     CUresult r = enc(map,
                      elt == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
@@ -188,8 +189,9 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
 
     const int64_t rows = (int64_t)num_pages * Hk * page_size;
     CUtensorMap kmap, vmap;
-    if (encode_kv_map(&kmap, k_pages, kv_dtype, head_dim, rows) != GQA_OK ||
-        encode_kv_map(&vmap, v_pages, kv_dtype, head_dim, rows) != GQA_OK)
+    const int box_rows = decode_tile_tokens(kv_dtype, page_size);
+    if (encode_kv_map(&kmap, k_pages, kv_dtype, head_dim, rows, box_rows) != GQA_OK ||
+        encode_kv_map(&vmap, v_pages, kv_dtype, head_dim, rows, box_rows) != GQA_OK)
         return GQA_ERR_LAUNCH;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -260,8 +262,8 @@ int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
     const int T = 128 / g;
     const int64_t rows = (int64_t)num_pages * Hk * page_size;
     CUtensorMap kmap, vmap, qmap;
-    if (encode_kv_map(&kmap, k_pages, GQA_KV_BF16, head_dim, rows) != GQA_OK ||
-        encode_kv_map(&vmap, v_pages, GQA_KV_BF16, head_dim, rows) != GQA_OK ||
+    if (encode_kv_map(&kmap, k_pages, GQA_KV_BF16, head_dim, rows, 16) != GQA_OK ||
+        encode_kv_map(&vmap, v_pages, GQA_KV_BF16, head_dim, rows, 16) != GQA_OK ||
         encode_q_map(&qmap, q, total_q, Hq, head_dim, g, T) != GQA_OK)
         return GQA_ERR_LAUNCH;
     PrefillArgs a;

@@ -35,7 +35,6 @@ namespace {
 
 constexpr int kConsumerWarps = kStreamWorkersPerCta;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kTile = kDecodeTileTokens;  // tokens per pipeline stage
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -45,13 +44,16 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kRingSplit = 65536;
 constexpr int kRingBalanced = 98304;
 
-template <int D, bool FP8, int RING = kRingSplit>
+// TT = tokens per pipeline stage (one TMA box of TT rows of one page and kv head): 16,
+// or 32 for e4m3 KV on pages of 32+ tokens (the fp8 tile then carries as many bytes as
+// a bf16 one, and two independent 16-token halves per softmax step).
+template <int D, bool FP8, int RING = kRingSplit, int TT = 16>
 struct Cfg {
     static constexpr int kElt = FP8 ? 1 : 2;
     static constexpr int kRowBytes = D * kElt;
     static constexpr int kBoxes = kRowBytes / 128;     // TMA boxes per tile row
     static constexpr int kBoxCols = 128 / kElt;        // elements per box row
-    static constexpr int kTileBytes = kTile * kRowBytes;
+    static constexpr int kTileBytes = TT * kRowBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kStagesRaw = RING / kStageBytes;
     static constexpr int kStages = kStagesRaw < 4 ? 4 : (kStagesRaw > 32 ? 32 : kStagesRaw);
@@ -67,9 +69,9 @@ struct TileRec {
     long long f; // flat tile index
 };
 
-template <int D, bool FP8, int RING = kRingSplit>
+template <int D, bool FP8, int RING = kRingSplit, int TT = 16>
 struct alignas(1024) Smem {
-    using C = Cfg<D, FP8, RING>;
+    using C = Cfg<D, FP8, RING, TT>;
     uint8_t tiles[C::kStages][2][C::kTileBytes];
     uint64_t full[C::kStages];
     uint64_t empty[C::kStages];
@@ -79,9 +81,11 @@ struct alignas(1024) Smem {
     int abort_flag;
 };
 
-// Byte offset of (row r, byte cb of the row; cb a multiple of 16) in a swizzled tile.
+// Byte offset of (row r, byte cb of the row; cb a multiple of 16) in a swizzled tile of
+// TT rows.
+template <int TT>
 __device__ __forceinline__ uint32_t swz(int r, int cb) {
-    return (uint32_t)((cb >> 7) * (kTile * 128) + r * 128 + ((((cb >> 4) & 7) ^ (r & 7)) << 4));
+    return (uint32_t)((cb >> 7) * (TT * 128) + r * 128 + ((((cb >> 4) & 7) ^ (r & 7)) << 4));
 }
 
 __device__ __forceinline__ void consumer_bar() {
@@ -100,9 +104,10 @@ __device__ __forceinline__ int clamp_len(int L, int Lmax, int *err) {
 // q fragments, the running max / sum per head, and O^T accumulators.
 //   fragment lane (gq = lane / 4, cq = lane % 4) holds heads 8*nt + 2*cq (+1) and, for
 //   dim tile dt, dims dim0(dt) and dim1(dt).
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, int TT>
 struct WarpAttn {
     static constexpr int KT = D / 16;
+    static constexpr int MT = TT / 16;  // 16-token halves of a tile
     uint32_t qf[NT][KT][2];
     float qmul;  // fp8 path: power-of-two prescale bringing q into f16 range
     float o[NT][KT][4];
@@ -181,94 +186,114 @@ struct WarpAttn {
         }
     }
 
-    // Fold one 16-token tile (valid tokens first, rows past them ignored) into the state.
+    // Fold one TT-token tile (valid tokens first, rows past them ignored) into the state.
     __device__ __forceinline__ void tile(uint8_t *kt, uint8_t *vt, int valid, float scale_log2,
                                          float ksc, float vsc, int lane) {
-        using C = Cfg<D, FP8>;
+        using C = Cfg<D, FP8, kRingSplit, TT>;
         const int gq = lane >> 2;
-        if (valid < kTile) {
+        if (valid < TT) {
             // Rows past the end of the sequence may hold anything (even NaN): zero the V
             // rows so 0-weight tokens contribute exactly 0; K rows are masked below.
             constexpr int kChunksPerRow = C::kRowBytes / 16;
-            for (int e = lane; e < (kTile - valid) * kChunksPerRow; e += 32) {
+            for (int e = lane; e < (TT - valid) * kChunksPerRow; e += 32) {
                 const int r = valid + e / kChunksPerRow, cb = (e % kChunksPerRow) * 16;
-                *reinterpret_cast<uint4 *>(vt + swz(r, cb)) = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(vt + swz<TT>(r, cb)) = make_uint4(0u, 0u, 0u, 0u);
             }
             __syncwarp();
         }
         const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
 
-        // ---- scores S^T[token][head] = K q^T
-        float s[NT][4];
+        // ---- scores S^T[token][head] = K q^T, per 16-token half
+        float s[MT][NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
         if (!FP8) {
-            const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-            for (int ks = 0; ks < KT; ++ks) {
-                uint32_t af[4];
-                ldsm_x4(af, kbase + swz(r, (ks * 16 + (lane >> 4) * 8) * 2));
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r = (lane & 7) + ((lane >> 3) & 1) * 8 + 16 * mt;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16(s[nt], af, qf[nt][ks][0], qf[nt][ks][1]);
+                for (int ks = 0; ks < KT; ++ks) {
+                    uint32_t af[4];
+                    ldsm_x4(af, kbase + swz<TT>(r, (ks * 16 + (lane >> 4) * 8) * 2));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(s[mt][nt], af, qf[nt][ks][0], qf[nt][ks][1]);
+                }
             }
         } else {
             // One ldmatrix.x4 over 32 fp8 dims serves two k steps; the k order inside a
             // step is permuted identically for K (here) and q (qf), which leaves each dot
             // product unchanged.
             const int j = lane >> 3;
-            const int r = (lane & 7) + (j & 1) * 8;
 #pragma unroll
-            for (int kp = 0; kp < D / 32; ++kp) {
-                uint32_t raw[4];
-                ldsm_x4(raw, kbase + swz(r, 32 * kp + (j >> 1) * 16));
-                uint32_t a0[4] = {e4m3x2_to_f16x2(raw[0] & 0xffff), e4m3x2_to_f16x2(raw[1] & 0xffff),
-                                  e4m3x2_to_f16x2(raw[0] >> 16), e4m3x2_to_f16x2(raw[1] >> 16)};
-                uint32_t a1[4] = {e4m3x2_to_f16x2(raw[2] & 0xffff), e4m3x2_to_f16x2(raw[3] & 0xffff),
-                                  e4m3x2_to_f16x2(raw[2] >> 16), e4m3x2_to_f16x2(raw[3] >> 16)};
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r = (lane & 7) + (j & 1) * 8 + 16 * mt;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_f16(s[nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-                    mma_f16(s[nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                for (int kp = 0; kp < D / 32; ++kp) {
+                    uint32_t raw[4];
+                    ldsm_x4(raw, kbase + swz<TT>(r, 32 * kp + (j >> 1) * 16));
+                    uint32_t a0[4] = {e4m3x2_to_f16x2(raw[0] & 0xffff), e4m3x2_to_f16x2(raw[1] & 0xffff),
+                                      e4m3x2_to_f16x2(raw[0] >> 16), e4m3x2_to_f16x2(raw[1] >> 16)};
+                    uint32_t a1[4] = {e4m3x2_to_f16x2(raw[2] & 0xffff), e4m3x2_to_f16x2(raw[3] & 0xffff),
+                                      e4m3x2_to_f16x2(raw[2] >> 16), e4m3x2_to_f16x2(raw[3] >> 16)};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_f16(s[mt][nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
+                        mma_f16(s[mt][nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                    }
                 }
             }
         }
 
-        // ---- online softmax (exp2 domain), per packed head column
+        // ---- online softmax (exp2 domain) over the tile, per packed head column
         const float kmul = FP8 ? scale_log2 * ksc / qmul : scale_log2;
-        const bool v0 = gq < valid, v1 = gq + 8 < valid;
-        uint32_t pb[NT][2], pbl[NT][2];
+        uint32_t pb[MT][NT][2], pbl[MT][NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float p[4], alpha[2];
+            float p[MT][4], alpha[2];
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
-                const float x0 = v0 ? s[nt][jj] * kmul : -INFINITY;
-                const float x1 = v1 ? s[nt][jj + 2] * kmul : -INFINITY;
-                float mx = fmaxf(x0, x1);
+                float x[MT][2];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    x[mt][0] = (16 * mt + gq < valid) ? s[mt][nt][jj] * kmul : -INFINITY;
+                    x[mt][1] = (16 * mt + gq + 8 < valid) ? s[mt][nt][jj + 2] * kmul : -INFINITY;
+                    mx = fmaxf(mx, fmaxf(x[mt][0], x[mt][1]));
+                }
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
                 const float mnew = fmaxf(m[nt][jj], mx);
                 const float mref = mnew == -INFINITY ? 0.f : mnew;
                 alpha[jj] = fast_exp2(m[nt][jj] - mref);
-                p[jj] = fast_exp2(x0 - mref);
-                p[jj + 2] = fast_exp2(x1 - mref);
-                l[nt][jj] = l[nt][jj] * alpha[jj] + p[jj] + p[jj + 2];
+                float sum = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    p[mt][jj] = fast_exp2(x[mt][0] - mref);
+                    p[mt][jj + 2] = fast_exp2(x[mt][1] - mref);
+                    sum += p[mt][jj] + p[mt][jj + 2];
+                }
+                l[nt][jj] = l[nt][jj] * alpha[jj] + sum;
                 m[nt][jj] = mnew;
             }
-            if (!FP8) {
-                // P as a bf16 value plus its bf16 residual: O += V^T P_hi^T + V^T P_lo^T keeps
-                // the weights at ~16 bits (one bf16 P would cost up to 2^-9 per weight).
-                uint32_t h0, l0, h1, l1;
-                split_bf16x2(p[0], p[1], h0, l0);
-                split_bf16x2(p[2], p[3], h1, l1);
-                pb[nt][0] = movmatrix_trans(h0);
-                pb[nt][1] = movmatrix_trans(h1);
-                pbl[nt][0] = movmatrix_trans(l0);
-                pbl[nt][1] = movmatrix_trans(l1);
-            } else {
-                pb[nt][0] = movmatrix_trans(pack_f16(p[0], p[1]));
-                pb[nt][1] = movmatrix_trans(pack_f16(p[2], p[3]));
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                if (!FP8) {
+                    // P as a bf16 value plus its bf16 residual: O += V^T P_hi^T + V^T P_lo^T
+                    // keeps the weights at ~16 bits (one bf16 P costs up to 2^-9 per weight).
+                    uint32_t h0, l0, h1, l1;
+                    split_bf16x2(p[mt][0], p[mt][1], h0, l0);
+                    split_bf16x2(p[mt][2], p[mt][3], h1, l1);
+                    pb[mt][nt][0] = movmatrix_trans(h0);
+                    pb[mt][nt][1] = movmatrix_trans(h1);
+                    pbl[mt][nt][0] = movmatrix_trans(l0);
+                    pbl[mt][nt][1] = movmatrix_trans(l1);
+                } else {
+                    pb[mt][nt][0] = movmatrix_trans(pack_f16(p[mt][0], p[mt][1]));
+                    pb[mt][nt][1] = movmatrix_trans(pack_f16(p[mt][2], p[mt][3]));
+                }
             }
 #pragma unroll
             for (int dt = 0; dt < KT; ++dt) {
@@ -282,43 +307,56 @@ struct WarpAttn {
         // ---- O^T[dim][head] += V^T P^T
         if (!FP8) {
             const int j = lane >> 3;
-            const int r = (lane & 7) + (j >> 1) * 8;
 #pragma unroll
-            for (int dt = 0; dt < KT; ++dt) {
-                uint32_t af[4];
-                ldsm_x4_trans(af, vbase + swz(r, (dt * 16 + (j & 1) * 8) * 2));
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r = (lane & 7) + (j >> 1) * 8 + 16 * mt;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_bf16(o[nt][dt], af, pb[nt][0], pb[nt][1]);
-                    mma_bf16(o[nt][dt], af, pbl[nt][0], pbl[nt][1]);
+                for (int dt = 0; dt < KT; ++dt) {
+                    uint32_t af[4];
+                    ldsm_x4_trans(af, vbase + swz<TT>(r, (dt * 16 + (j & 1) * 8) * 2));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_bf16(o[nt][dt], af, pb[mt][nt][0], pb[mt][nt][1]);
+                        mma_bf16(o[nt][dt], af, pbl[mt][nt][0], pbl[mt][nt][1]);
+                    }
                 }
             }
         } else {
             // fp8 V: plain ldmatrix gives each lane 4 consecutive dims of one token;
             // after conversion, movmatrix transposes 8x8 blocks into the A layout (dims
             // permuted within each 16-dim tile; dim0/dim1 undo it when O is written).
+            // The tile's P.V is summed apart and scaled once by the tile's V scale.
+            float pv[NT][KT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt) pv[nt][dt][0] = pv[nt][dt][1] = pv[nt][dt][2] = pv[nt][dt][3] = 0.f;
             const int j = lane >> 3;
-            const int r = (lane & 7) + (j & 1) * 8;
 #pragma unroll
-            for (int qd = 0; qd < D / 32; ++qd) {
-                uint32_t raw[4];
-                ldsm_x4(raw, vbase + swz(r, 32 * qd + (j >> 1) * 16));
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r = (lane & 7) + (j & 1) * 8 + 16 * mt;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t lo_t = raw[2 * h], hi_t = raw[2 * h + 1];  // tokens 0-7 / 8-15
-                    uint32_t af[4] = {movmatrix_trans(e4m3x2_to_f16x2(lo_t & 0xffff)),
-                                      movmatrix_trans(e4m3x2_to_f16x2(lo_t >> 16)),
-                                      movmatrix_trans(e4m3x2_to_f16x2(hi_t & 0xffff)),
-                                      movmatrix_trans(e4m3x2_to_f16x2(hi_t >> 16))};
+                for (int qd = 0; qd < D / 32; ++qd) {
+                    uint32_t raw[4];
+                    ldsm_x4(raw, vbase + swz<TT>(r, 32 * qd + (j >> 1) * 16));
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        float pv[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_f16(pv, af, pb[nt][0], pb[nt][1]);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t lo_t = raw[2 * h], hi_t = raw[2 * h + 1];  // tokens 0-7 / 8-15
+                        uint32_t af[4] = {movmatrix_trans(e4m3x2_to_f16x2(lo_t & 0xffff)),
+                                          movmatrix_trans(e4m3x2_to_f16x2(lo_t >> 16)),
+                                          movmatrix_trans(e4m3x2_to_f16x2(hi_t & 0xffff)),
+                                          movmatrix_trans(e4m3x2_to_f16x2(hi_t >> 16))};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) o[nt][2 * qd + h][e] += vsc * pv[e];
+                        for (int nt = 0; nt < NT; ++nt) mma_f16(pv[nt][2 * qd + h], af, pb[mt][nt][0], pb[mt][nt][1]);
                     }
                 }
             }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[nt][dt][e] += vsc * pv[nt][dt][e];
         }
     }
 
@@ -338,16 +376,17 @@ struct WarpAttn {
 };
 
 // ========================================================================== split schedule
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, int TT>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const DecodeArgs a, const int heads_per_cta, const int head_chunks) {
-    using C = Cfg<D, FP8>;
+    using C = Cfg<D, FP8, kRingSplit, TT>;
+    constexpr int kTile = TT;
     constexpr int S = C::kStages;
     constexpr int KT = D / 16;
     extern __shared__ uint8_t smem_raw[];
-    Smem<D, FP8> &sm = *reinterpret_cast<Smem<D, FP8> *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using SMT = Smem<D, FP8, kRingSplit, TT>;
+    SMT &sm = *reinterpret_cast<SMT *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x;
@@ -450,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 
     // -------------------------------------------------------------------- consumers
     const int gq = lane >> 2, cq = lane & 3;
-    WarpAttn<D, NT, FP8> st;
+    WarpAttn<D, NT, FP8, TT> st;
     st.load_q(reinterpret_cast<const __nv_bfloat16 *>(a.q) + ((size_t)b * a.Hq + head_lo) * D, nh, lane);
     st.reset();
     const float scale_log2 = a.scale * kLog2e;
@@ -488,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         const int h0 = nt * 8 + 2 * cq;
 #pragma unroll
         for (int dt = 0; dt < KT; ++dt) {
-            const int d0 = WarpAttn<D, NT, FP8>::dim0(dt, gq), d1 = WarpAttn<D, NT, FP8>::dim1(dt, gq);
+            const int d0 = WarpAttn<D, NT, FP8, TT>::dim0(dt, gq), d1 = WarpAttn<D, NT, FP8, TT>::dim1(dt, gq);
             float *w = red_o + (size_t)(warp * HW + h0) * RS;
             w[d0] = st.o[nt][dt][0];
             w[RS + d0] = st.o[nt][dt][1];
@@ -644,14 +683,15 @@ __device__ __forceinline__ void merge_pieces(const float *pieces, long long wfir
     }
 }
 
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, int TT>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     decode_sk_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const DecodeArgs a,
                      const int heads_per_cta, const int head_chunks) {
-    using C = Cfg<D, FP8, kRingBalanced>;
-    using SM = Smem<D, FP8, kRingBalanced>;
-    using WA = WarpAttn<D, NT, FP8>;
+    using C = Cfg<D, FP8, kRingBalanced, TT>;
+    using SM = Smem<D, FP8, kRingBalanced, TT>;
+    using WA = WarpAttn<D, NT, FP8, TT>;
+    constexpr int kTile = TT;
     constexpr int S = C::kStages;
     constexpr int SW = S / kConsumerWarps;  // stages per worker
     constexpr int KT = D / 16;
@@ -874,29 +914,31 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     }
 }
 
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, int TT>
 cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
                      cudaStream_t stream) {
     static_assert(sizeof(float) * kConsumerWarps * 8 * NT * (D + 6) <=
-                      sizeof(uint8_t) * Cfg<D, FP8>::kStages * 2 * Cfg<D, FP8>::kTileBytes,
+                      sizeof(uint8_t) * Cfg<D, FP8, kRingSplit, TT>::kStages * 2 *
+                          Cfg<D, FP8, kRingSplit, TT>::kTileBytes,
                   "reduction area must fit in the stage ring");
     const int g = a.Hq / a.Hk;
     const int hpc = a.pack_gqa ? (g < 8 * NT ? g : 8 * NT) : 1;
     const int chunks = (g + hpc - 1) / hpc;
     if (a.stream_k) {
-        const size_t smem = sizeof(Smem<D, FP8, kRingBalanced>) + 1024 + sizeof(int) * (size_t)(a.B + 1);
-        cudaError_t e = cudaFuncSetAttribute(decode_sk_kernel<D, NT, FP8>,
+        const size_t smem =
+            sizeof(Smem<D, FP8, kRingBalanced, TT>) + 1024 + sizeof(int) * (size_t)(a.B + 1);
+        cudaError_t e = cudaFuncSetAttribute(decode_sk_kernel<D, NT, FP8, TT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_sk_kernel<D, NT, FP8><<<a.grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
+        decode_sk_kernel<D, NT, FP8, TT><<<a.grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
         return cudaGetLastError();
     }
-    const size_t smem = sizeof(Smem<D, FP8>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8>,
+    const size_t smem = sizeof(Smem<D, FP8, kRingSplit, TT>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8, TT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.num_splits, a.Hk * chunks, a.B);
-    decode_kernel<D, NT, FP8><<<grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
+    decode_kernel<D, NT, FP8, TT><<<grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
     return cudaGetLastError();
 }
 
@@ -907,14 +949,17 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &kmap, const CU
     const int g = a.Hq / a.Hk;
     const bool wide = a.pack_gqa && g > 8;
     if (a.kv_dtype == GQA_KV_FP8_E4M3) {
-        return wide ? launch_t<128, 2, true>(a, kmap, vmap, stream)
-                    : launch_t<128, 1, true>(a, kmap, vmap, stream);
+        if (decode_tile_tokens(a.kv_dtype, a.P) == 32)
+            return wide ? launch_t<128, 2, true, 32>(a, kmap, vmap, stream)
+                        : launch_t<128, 1, true, 32>(a, kmap, vmap, stream);
+        return wide ? launch_t<128, 2, true, 16>(a, kmap, vmap, stream)
+                    : launch_t<128, 1, true, 16>(a, kmap, vmap, stream);
     }
     if (a.D == 128)
-        return wide ? launch_t<128, 2, false>(a, kmap, vmap, stream)
-                    : launch_t<128, 1, false>(a, kmap, vmap, stream);
-    return wide ? launch_t<64, 2, false>(a, kmap, vmap, stream)
-                : launch_t<64, 1, false>(a, kmap, vmap, stream);
+        return wide ? launch_t<128, 2, false, 16>(a, kmap, vmap, stream)
+                    : launch_t<128, 1, false, 16>(a, kmap, vmap, stream);
+    return wide ? launch_t<64, 2, false, 16>(a, kmap, vmap, stream)
+                : launch_t<64, 1, false, 16>(a, kmap, vmap, stream);
 }
 
 }  // namespace gqa

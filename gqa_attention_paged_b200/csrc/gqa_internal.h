@@ -79,7 +79,10 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap,
                            const CUtensorMap &vmap, const CUtensorMap &qmap,
                            cudaStream_t stream);
 
-// Box sizes the tensor maps must be encoded with.
-constexpr int kDecodeTileTokens = 16;
+// Tokens per decode pipeline stage (the TMA box height of the KV tensor maps): 32 for
+// e4m3 KV on pages of at least 32 tokens, else 16.
+inline int decode_tile_tokens(int kv_dtype, int page_size) {
+    return (kv_dtype == 1 && page_size >= 32) ? 32 : 16;
+}
 
 }  // namespace gqa

@@ -301,21 +301,26 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             // reading it twice keeps the row's 128 scores out of the register file).
             const int nvis = lim - j * kN + 1;  // keys of this tile the row may see
             float mx = -INFINITY, mx1 = -INFINITY;
+            {
+                // all four loads in flight before one wait: tensor-memory reads are cheap,
+                // their round trips are not
+                uint32_t sa[4][32];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t sa[32];
-                tmem_ld32(tS + 32 * cc, sa);
+                for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, sa[cc]);
                 tmem_wait_ld();
-                if (nvis >= 32 * cc + 32) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        mx = fmaxf(mx, __uint_as_float(sa[e]));
-                        mx1 = fmaxf(mx1, __uint_as_float(sa[e + 1]));
+                for (int cc = 0; cc < 4; ++cc) {
+                    if (nvis >= 32 * cc + 32) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            mx = fmaxf(mx, __uint_as_float(sa[cc][e]));
+                            mx1 = fmaxf(mx1, __uint_as_float(sa[cc][e + 1]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            mx = fmaxf(mx, (32 * cc + e < nvis) ? __uint_as_float(sa[cc][e]) : -INFINITY);
                     }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        mx = fmaxf(mx, (32 * cc + e < nvis) ? __uint_as_float(sa[e]) : -INFINITY);
                 }
             }
             mx = fmaxf(mx, mx1);
@@ -371,7 +376,6 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     sum2 = f2_add(sum2, pp);
                     __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                     hi[e] = *reinterpret_cast<uint32_t *>(&h);
-                    // residual: p - float(bf16(p)), exact in fp32
                     const unsigned long long hf = f2_pack(__uint_as_float(hi[e] << 16),
                                                           __uint_as_float(hi[e] & 0xffff0000u));
                     float r0, r1;

@@ -118,6 +118,21 @@ def test_long70b_decode_fp8(S):
     assert np.max(np.abs(out - ref_o)) <= 5e-2, f"fp8 vs bf16 oracle: {err_report(out, ref_o)}"
 
 
+@pytest.mark.parametrize("P", [16, 32, 64])
+@pytest.mark.parametrize("Hq,Hk", [(32, 8), (64, 8), (8, 8)])
+def test_fp8_page_sizes_and_ragged_tiles(P, Hq, Hk):
+    """e4m3 KV takes 32-token tiles on pages of 32+ tokens: lengths that end inside either
+    16-token half of a tile, exactly on a tile edge, empty, and longer than a page."""
+    lens = [1, 15, 16, 17, 31, 32, 33, 0, 63, 200]
+    case = inputs.make_decode_case(len(lens), Hq, Hk, 128, P, lens, seed=P + Hq,
+                                   kv_dtype="fp8_e4m3", outlier_p=0.01)
+    ref_o, ref_l = oracle_decode(case)
+    dev = to_dev(case)
+    for S, pack in ((0, True), (1, True), (3, True), (1, False)):
+        out, lse = run_decode(case, num_splits=S, pack_gqa=pack, dev=dev)
+        check(out, lse, ref_o, ref_l, what=f"fp8 P={P} Hq={Hq} S={S} pack={pack}")
+
+
 @pytest.mark.parametrize("Hq,Hk,D,P", [(8, 8, 64, 16), (8, 1, 64, 32), (32, 1, 128, 16),
                                        (12, 4, 128, 64), (40, 8, 128, 16), (16, 2, 64, 64)])
 def test_head_layouts_mha_mqa_and_odd_groups(Hq, Hk, D, P):
