@@ -14,19 +14,24 @@
 // softmax in registers, P written back into tensor memory over S, and O += P V on
 // tcgen05 with P read from tensor memory.
 //
-// Warp roles (320 threads):
-//   warp 0     TMA producer: both Q tiles (3-D map over [total_q][Hq][D]), then K and V
-//              tiles, 16 keys per copy, gathered page by page through the page table.
-//   warp 1     allocates all 512 tensor-memory columns (S0, S1, O0, O1) and issues the
-//              MMAs from one thread in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so the
-//              tensor core works on one query tile while the other one's softmax runs.
-//   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1; a thread owns one row
-//              (one tensor-memory lane).
-// P is stored as a bf16 value plus its bf16 residual and O += P_hi V + P_lo V, which
-// keeps the probabilities at ~16 significant bits (a single bf16 P loses up to 2^-9 of
-// each weight, visible as ~5e-3 errors in short rows whose terms cancel).
+// Warp roles (384 threads, three warpgroups):
+//   warp 0      TMA producer: both Q tiles (3-D map over [total_q][Hq][D]), then K and V
+//               tiles, 16 keys per copy, gathered page by page through the page table.
+//   warp 1      allocates all 512 tensor-memory columns (S0, S1, O0, O1) and issues the
+//               MMAs from one thread in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so the
+//               tensor core works on one query tile while the other one's softmax runs.
+//   warps 2-3   convert each V tile in place from bf16 to f16 (zeroing keys past the
+//               sequence first), unless a value is beyond the f16 range.
+//   warps 4-7   softmax of query tile 0, warps 8-11 of query tile 1; a thread owns one
+//               row (one tensor-memory lane) and holds its 128 scores in registers.
+// The softmax warpgroups take most of the register file (setmaxnreg).
+//
+// P precision: P is written as f16 (11 significant bits) and multiplied with the f16
+// copy of V, so O += P V keeps each weight to 2^-12 relative.  A V tile holding a value
+// of magnitude 2^16 or more (or Inf / NaN) stays bf16; for that tile P is written as a
+// bf16 value plus its bf16 residual and O += P_hi V + P_lo V (~16 significant bits).
 // The running max is only moved when a row's max grows by more than 2^8, so O is
-// rescaled rarely; the final O / l is exact for any reference max.
+// rescaled rarely and P stays below 2^8; the final O / l is exact for any reference.
 // Every wait is bounded; on expiry the kernel records GQA_ERR_TIMEOUT, finishes its
 // outstanding copies and MMAs (bounded), frees its tensor memory and returns.
 #include "gqa_device.cuh"
@@ -39,8 +44,9 @@ constexpr int kM = 128;                // packed query rows per query tile
 constexpr int kQT = 2;                 // query tiles per CTA
 constexpr int kN = 128;                // keys per KV tile
 constexpr int kD = 128;                // head dim
-constexpr int kStages = 2;             // K/V ring depth
-constexpr int kThreadsP = 320;
+constexpr int kKStages = 2;            // K ring depth
+constexpr int kVStages = 3;            // V ring depth (a V tile also waits for its conversion)
+constexpr int kThreadsP = 384;
 constexpr int kHalfBytes = kM * 128;   // one 64-column (128-byte) half of a 128-row tile
 constexpr int kTileBytesP = 2 * kHalfBytes;
 constexpr int kChunk = 16;             // keys per TMA copy (one box)
@@ -49,21 +55,222 @@ constexpr float kLog2eP = 1.4426950408889634f;
 constexpr float kLn2P = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr unsigned kAll = 0xffffffffu;
+// Register split: warpgroup 0 (producer, MMA, converters) keeps 64 per thread, the two
+// softmax warpgroups take 216: 128*64 + 256*216 <= 384*168, the launch allocation.
+constexpr int kRegsSide = 64;
+constexpr int kRegsSoftmax = 216;
+static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreadsP * 168, "register split");
+constexpr int kConvThreads = 64;
+// |bf16 bits| at or above this (2^16, and Inf / NaN) does not convert to a finite f16
+constexpr uint32_t kF16Limit = 0x4780u;
 
 struct alignas(1024) PSmem {
     uint8_t q[kQT][kTileBytesP];
-    uint8_t k[kStages][kTileBytesP];
-    uint8_t v[kStages][kTileBytesP];
+    uint8_t k[kKStages][kTileBytesP];
+    uint8_t v[kVStages][kTileBytesP];
     uint64_t q_full;
-    uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    uint64_t k_full[kKStages], k_empty[kKStages];
+    uint64_t v_full[kVStages], v_ready[kVStages], v_empty[kVStages];
     uint64_t s_full[kQT], p_full[kQT], pv_done[kQT];
     uint64_t mma_done;
+    int v_bf16[kVStages];       // 1: the V tile stayed bf16 (a value out of f16 range)
+    int conv_ovf[kVStages][2];  // per converter warp: (tile + 1) * 2 + out-of-range flag
     uint32_t tmem_base;
 };
+
+static_assert(sizeof(PSmem) + 1024 <= 227 * 1024, "shared memory per CTA");
 
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);
     return !__any_sync(kAll, !ok);
+}
+
+// KV row (in the [num_pages*Hk*P][D] view) of the 16-key chunk `lane` of KV tile j, or -1
+// for lanes past the 8 chunks, keys at or past L, and out-of-range page entries (which
+// set GQA_ERR_BAD_PAGE).
+__device__ __forceinline__ int kv_chunk_row(const PrefillArgs &a, const int32_t *pt, int j,
+                                            int lane, int kvh, int L) {
+    const int key0 = j * kN + kChunk * lane;
+    if (lane >= kN / kChunk || key0 >= L) return -1;
+    const int phys = __ldg(pt + key0 / a.P);
+    if (phys < 0 || phys >= a.num_pages) {
+        set_error(a.err, GQA_ERR_BAD_PAGE);
+        return -1;
+    }
+    return (phys * a.Hk + kvh) * a.P + key0 % a.P;
+}
+
+// Softmax warpgroup of query tile (warp - 4) / 4: online softmax over the score tiles in
+// tensor memory, P written back over S, final O / l and LSE to global memory.
+__device__ __forceinline__ void softmax_role(PSmem &sm, const PrefillArgs &a, const uint32_t tmem,
+                                             const int warp, const int lane, const int (&n_kv_q)[kQT],
+                                             const int b, const int kvh, const int g, const int q0,
+                                             const int Lq, const int i0, const int T, const int L) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int q = (warp - 4) / 4;  // query tile
+    const int quad = warp & 3;     // tensor-memory lane quadrant this warp may access
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + 128 * q + lane_off, tO = tmem + 256 + 128 * q + lane_off;
+    const int nk = n_kv_q[q];
+    const int ntok = min(T, Lq - (i0 + q * T));
+    const bool valid_row = row < ntok * g;
+    const int tok = i0 + q * T + row / g;
+    const int hh = row % g;
+    const int lim = a.causal ? min(L - Lq + tok, L - 1) : L - 1;  // last visible key
+    const float c = a.scale * kLog2eP;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+        const int stage = j % kVStages;
+        if (!wait_all(&sm.s_full[q], j & 1)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after_sync();
+        // the row's 128 scores: all four loads in flight before one wait
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, sr[cc]);
+        tmem_wait_ld();
+        const int nvis = lim - j * kN + 1;  // keys of this tile the row may see
+        if (nvis < kN) {  // diagonal / tail tile: scores past nvis -> -inf
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (32 * cc + e >= nvis) sr[cc][e] = __float_as_uint(-INFINITY);
+        }
+        float mx;
+        {
+            float m4[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float t = fmax3(__uint_as_float(sr[cc][0]), __uint_as_float(sr[cc][1]),
+                                __uint_as_float(sr[cc][2]));
+#pragma unroll
+                for (int e = 3; e < 31; e += 2)
+                    t = fmax3(t, __uint_as_float(sr[cc][e]), __uint_as_float(sr[cc][e + 1]));
+                m4[cc] = fmaxf(t, __uint_as_float(sr[cc][31]));
+            }
+            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+        mx *= c;  // c > 0: the max commutes with the scale
+        const bool need = mx > m_ref + kRescaleThreshold;
+        const float new_ref = need ? mx : m_ref;
+        const float mref0 = new_ref == -INFINITY ? 0.f : new_ref;
+        const float alpha = ex2_approx(m_ref - mref0);
+
+        if (j > 0 && __any_sync(kAll, need)) {
+            // O must not be touched while PV(j-1) still accumulates into it
+            if (!wait_all(&sm.pv_done[q], (j - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(tO + 32 * cc, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st32(tO + 32 * cc, o);
+            }
+        }
+        // the form P takes depends on whether this V tile became f16
+        if (!wait_all(&sm.v_ready[stage], (j / kVStages) & 1)) {
+            ok = false;
+            break;
+        }
+        const bool vbf = sm.v_bf16[stage] != 0;
+        // P = 2^(s*c - ref), written over S chunk by chunk: the 32 keys of chunk cc
+        // (columns [32cc, 32cc+32) of S) become 16 columns of value pairs, plus 16 of
+        // residual pairs when the tile stayed bf16.  Keys go in pairs through the
+        // paired fp32 instructions.
+        const unsigned long long c2 = f2_pack(c, c), nref2 = f2_pack(-mref0, -mref0);
+        unsigned long long sum2 = 0ull;  // (0.f, 0.f)
+        if (!vbf) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cc][2 * e]),
+                                             __uint_as_float(sr[cc][2 * e + 1])),
+                                     c2, nref2),
+                              x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    sum2 = f2_add(sum2, f2_pack(p0, p1));
+                    pk[e] = pack_f16(p0, p1);
+                }
+                tmem_st16(tS + 32 * cc, pk);
+            }
+        } else {
+            const unsigned long long neg1 = f2_pack(-1.f, -1.f);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cc][2 * e]),
+                                             __uint_as_float(sr[cc][2 * e + 1])),
+                                     c2, nref2),
+                              x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    const unsigned long long pp = f2_pack(p0, p1);
+                    sum2 = f2_add(sum2, pp);
+                    hi[e] = pack_bf16(p0, p1);
+                    const unsigned long long hf = f2_pack(__uint_as_float(hi[e] << 16),
+                                                          __uint_as_float(hi[e] & 0xffff0000u));
+                    float r0, r1;
+                    f2_unpack(f2_fma(hf, neg1, pp), r0, r1);
+                    lo[e] = pack_bf16(r0, r1);
+                }
+                tmem_st16(tS + 32 * cc, hi);
+                tmem_st16(tS + 32 * cc + 16, lo);
+            }
+        }
+        float sum, sum_hi;
+        f2_unpack(sum2, sum, sum_hi);
+        sum += sum_hi;
+        tmem_wait_st();
+        l = l * alpha + sum;
+        m_ref = new_ref;
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[q]);
+    }
+    if (nk > 0 && ok && wait_all(&sm.pv_done[q], (nk - 1) & 1)) {
+        tc_fence_after_sync();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) +
+                             ((size_t)(q0 + tok) * a.Hq + kvh * g + hh) * kD;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * cc, o);
+            tmem_wait_ld();
+            if (valid_row) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    uint4 w;
+                    w.x = pack_bf16(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+                    w.y = pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+                    w.z = pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+                    w.w = pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+                    *reinterpret_cast<uint4 *>(dst + 32 * cc + e) = w;
+                }
+            }
+        }
+        if (valid_row && a.lse)
+            a.lse[(size_t)(q0 + tok) * a.Hq + kvh * g + hh] =
+                l > 0.f ? (m_ref + __log2f(l)) * kLn2P : -INFINITY;
+    } else if (nk > 0 && lane == 0) {
+        set_error(a.err, GQA_ERR_TIMEOUT);
+    }
 }
 
 __global__ void __launch_bounds__(kThreadsP, 1)
@@ -101,10 +308,14 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(&sm.v_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.v_ready[s], 2);
+            mbar_init(&sm.v_empty[s], 1);
         }
         for (int q = 0; q < kQT; ++q) {
             mbar_init(&sm.s_full[q], 1);
@@ -112,6 +323,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             mbar_init(&sm.pv_done[q], 1);
         }
         mbar_init(&sm.mma_done, 1);
+        for (int s = 0; s < kVStages; ++s) sm.conv_ovf[s][0] = sm.conv_ovf[s][1] = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -124,6 +336,12 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     tc_fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
 
+    if (warp >= 4) {
+        regs_acquire<kRegsSoftmax>();
+        softmax_role(sm, a, tmem, warp, lane, n_kv_q, b, kvh, g, q0, Lq, i0, T, L);
+    } else {
+    // every warp of warpgroup 0 gives its registers back at the same instruction
+    regs_release<kRegsSide>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         const uint64_t pol_kv = policy_evict_last();  // K/V are re-read by the other q tiles
@@ -138,56 +356,34 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                                 q0 + i0 + q * T, policy_evict_first());
         }
         const int32_t *pt = a.page_table + (size_t)b * a.pt_stride;
-        int issued = 0;
-        bool fail = false;
-        for (int j = 0; j < n_kv && !fail; ++j) {
-            const int stage = j % kStages, use = j / kStages;
-            const int key0 = j * kN + kChunk * lane;
-            int row = -1;
-            if (lane < kN / kChunk && key0 < L) {
-                const int phys = __ldg(pt + key0 / P);
-                if (phys >= 0 && phys < a.num_pages)
-                    row = (phys * a.Hk + kvh) * P + key0 % P;
-                else
-                    set_error(a.err, GQA_ERR_BAD_PAGE);
-            }
+        int issued_k = 0;
+        for (int j = 0; j < n_kv; ++j) {
+            const int row = kv_chunk_row(a, pt, j, lane, kvh, L);
             const unsigned mask = __ballot_sync(kAll, row >= 0);
-            int rows[kN / kChunk];
-#pragma unroll
-            for (int c = 0; c < kN / kChunk; ++c) rows[c] = __shfl_sync(kAll, row, c);
+            const int ks = j % kKStages, use = j / kKStages;
+            bool fail = false;
             if (lane == 0) {
-                if (use > 0 && !mbar_wait(&sm.kv_empty[stage], (use - 1) & 1)) {
+                if (use > 0 && !mbar_wait(&sm.k_empty[ks], (use - 1) & 1)) {
                     set_error(a.err, GQA_ERR_TIMEOUT);
                     fail = true;
                 } else {
-                    // K first: the S MMAs can start before V lands
-                    mbar_arrive_expect_tx(&sm.k_full[stage], __popc(mask) * 2 * kChunkBytes);
-#pragma unroll
-                    for (int c = 0; c < kN / kChunk; ++c)
-                        if ((mask >> c) & 1u)
-#pragma unroll
-                            for (int h = 0; h < 2; ++h)
-                                tma_load_2d(sm.k[stage] + h * kHalfBytes + c * kChunkBytes, &kmap,
-                                            &sm.k_full[stage], 64 * h, rows[c], pol_kv);
-                    mbar_arrive_expect_tx(&sm.v_full[stage], __popc(mask) * 2 * kChunkBytes);
-#pragma unroll
-                    for (int c = 0; c < kN / kChunk; ++c)
-                        if ((mask >> c) & 1u)
-#pragma unroll
-                            for (int h = 0; h < 2; ++h)
-                                tma_load_2d(sm.v[stage] + h * kHalfBytes + c * kChunkBytes, &vmap,
-                                            &sm.v_full[stage], 64 * h, rows[c], pol_kv);
-                    issued = j + 1;
+                    mbar_arrive_expect_tx(&sm.k_full[ks], __popc(mask) * 2 * kChunkBytes);
                 }
             }
-            fail = __shfl_sync(kAll, fail, 0);
+            if (__shfl_sync(kAll, fail, 0)) break;
+            if (row >= 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(sm.k[ks] + h * kHalfBytes + lane * kChunkBytes, &kmap,
+                                &sm.k_full[ks], 64 * h, row, pol_kv);
+            }
+            issued_k = j + 1;
         }
         if (lane == 0) {
-            // no copy may outlive the CTA: wait for the Q tiles and the last issued K/V tiles
+            // no copy may outlive the CTA: wait for the Q tiles and the last issued K tiles
             if (!mbar_wait(&sm.q_full, 0)) set_error(a.err, GQA_ERR_TIMEOUT);
-            for (int j = max(0, issued - kStages); j < issued; ++j)
-                if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1) ||
-                    !mbar_wait(&sm.v_full[j % kStages], (j / kStages) & 1)) {
+            for (int j = max(0, issued_k - kKStages); j < issued_k; ++j)
+                if (!mbar_wait(&sm.k_full[j % kKStages], (j / kKStages) & 1)) {
                     set_error(a.err, GQA_ERR_TIMEOUT);
                     break;
                 }
@@ -195,12 +391,13 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);   // Q, K both K-major
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, kD, 0, 1);   // P (TMEM), V MN-major
+        constexpr uint32_t idesc_pv16 = idesc_f16_f32(kM, kD, 0, 1);  // P (TMEM), V MN-major
+        constexpr uint32_t idesc_pvbf = idesc_bf16_f32(kM, kD, 0, 1);
         bool ok = wait_all(&sm.q_full, 0);
         // S_q(j) = Q_q K_j^T into tensor-memory columns [128 q, 128 q + 128)
         auto issue_s = [&](int q, int j) -> bool {
-            const int stage = j % kStages;
-            if (!wait_all(&sm.k_full[stage], (j / kStages) & 1)) return false;
+            const int stage = j % kKStages;
+            if (!wait_all(&sm.k_full[stage], (j / kKStages) & 1)) return false;
             tc_fence_after_sync();
             if (lane == 0) {
                 const uint32_t qa = smem_u32(sm.q[q]), ka = smem_u32(sm.k[stage]);
@@ -215,59 +412,51 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             __syncwarp();
             return true;
         };
-        // O_q += P_q(j) V_j with P_q(j) in S_q's columns: keys 32c..32c+31 as bf16 value
-        // pairs in columns [32c, 32c+16) and residual pairs in [32c+16, 32c+32)
+        // O_q += P_q(j) V_j with P_q(j) in S_q's columns: keys 32c..32c+31 as value pairs
+        // in columns [32c, 32c+16): f16 against the f16 V tile, or bf16 with the residual
+        // pairs in [32c+16, 32c+32) against a V tile that stayed bf16.
         auto issue_pv = [&](int q, int j) -> bool {
-            const int stage = j % kStages;
+            const int stage = j % kVStages;
             if (!wait_all(&sm.p_full[q], j & 1) ||
-                !wait_all(&sm.v_full[stage], (j / kStages) & 1))
+                !wait_all(&sm.v_ready[stage], (j / kVStages) & 1))
                 return false;
             tc_fence_after_sync();
+            const bool vbf = sm.v_bf16[stage] != 0;
             if (lane == 0) {
                 const uint32_t va = smem_u32(sm.v[stage]);
                 const uint32_t tp = tmem + 128 * q, to = tmem + 256 + 128 * q;
+                const uint32_t idesc = vbf ? idesc_pvbf : idesc_pv16;
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk)
                     tc_mma_ts(to, tp + 32 * (kk >> 1) + 8 * (kk & 1),
-                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc,
                               (j > 0 || kk > 0) ? 1u : 0u);
+                if (vbf) {
 #pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk)
-                    tc_mma_ts(to, tp + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
-                              smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv, 1u);
+                    for (int kk = 0; kk < kN / 16; ++kk)
+                        tc_mma_ts(to, tp + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
+                                  smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pvbf, 1u);
+                }
                 tc_commit(&sm.pv_done[q]);
             }
             __syncwarp();
             return true;
         };
+        // K tile j is released once the S MMAs that read it are done, V tile j once PV(j)
         for (int q = 0; q < kQT && ok; ++q)
             if (n_kv_q[q] > 0) ok = issue_s(q, 0);
+        if (ok && lane == 0 && n_kv > 0) tc_commit(&sm.k_empty[0]);
+        __syncwarp();
         for (int j = 0; j < n_kv && ok; ++j) {
-            const int stage = j % kStages;
-            if (j == n_kv - 1) {
-                // keys at or past L hold anything (even NaN): zero those V rows so their
-                // zero weights contribute exactly zero.
-                const int valid = L - j * kN;
-                if (valid < kN) {
-                    if (!wait_all(&sm.v_full[stage], (j / kStages) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    for (int e = lane; e < (kN - valid) * 16; e += 32) {
-                        const int r = valid + (e >> 4), c16 = e & 15;
-                        *reinterpret_cast<uint4 *>(sm.v[stage] + (c16 >> 3) * kHalfBytes + r * 128 +
-                                                   (c16 & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-            }
             for (int q = 0; q < kQT && ok; ++q) {
                 if (j >= n_kv_q[q]) continue;
                 ok = issue_pv(q, j);
                 if (ok && j + 1 < n_kv_q[q]) ok = issue_s(q, j + 1);
             }
-            if (ok && lane == 0) tc_commit(&sm.kv_empty[stage]);
+            if (ok && lane == 0) {
+                tc_commit(&sm.v_empty[j % kVStages]);
+                if (j + 1 < n_kv) tc_commit(&sm.k_empty[(j + 1) % kKStages]);
+            }
             __syncwarp();
         }
         if (!ok && lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
@@ -276,153 +465,123 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         __syncwarp();
         if (!wait_all(&sm.mma_done, 0) && lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
     } else {
-        // ------------------------------------------------------------ softmax warpgroups
-        const int q = (warp - 2) / 4;  // query tile
-        const int quad = warp & 3;     // tensor-memory lane quadrant this warp may access
-        const int row = quad * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tS = tmem + 128 * q + lane_off, tO = tmem + 256 + 128 * q + lane_off;
-        const int nk = n_kv_q[q];
-        const int ntok = min(T, Lq - (i0 + q * T));
-        const bool valid_row = row < ntok * g;
-        const int tok = i0 + q * T + row / g;
-        const int hh = row % g;
-        const int lim = a.causal ? min(L - Lq + tok, L - 1) : L - 1;  // last visible key
-        const float c = a.scale * kLog2eP;
-        float m_ref = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int j = 0; j < nk; ++j) {
-            if (!wait_all(&sm.s_full[q], j & 1)) {
-                ok = false;
+        // ------------------------------------------------------------ V loads + converters
+        // Warp 2 also copies the V tiles in (one lane per 16-key chunk): the first
+        // kVStages at once, then, after converting tile j, it waits for PV(j - 1) to free
+        // that tile's stage and loads tile j + kVStages - 1 into it.
+        const int cid = threadIdx.x - 64;  // 0..63
+        const int cw = warp - 2;
+        constexpr int kChunks16 = kTileBytesP / 16;  // 16-byte chunks of a V tile
+        const int32_t *pt = a.page_table + (size_t)b * a.pt_stride;
+        const uint64_t pol_kv = policy_evict_last();
+        int issued_v = 0;
+        auto load_v = [&](int jv) {
+            const int row = kv_chunk_row(a, pt, jv, lane, kvh, L);
+            const unsigned mask = __ballot_sync(kAll, row >= 0);
+            const int vs = jv % kVStages;
+            if (lane == 0) mbar_arrive_expect_tx(&sm.v_full[vs], __popc(mask) * 2 * kChunkBytes);
+            __syncwarp();
+            if (row >= 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(sm.v[vs] + h * kHalfBytes + lane * kChunkBytes, &vmap,
+                                &sm.v_full[vs], 64 * h, row, pol_kv);
+            }
+            issued_v = jv + 1;
+        };
+        if (cw == 0)
+            for (int jv = 0; jv < min(n_kv, kVStages); ++jv) load_v(jv);
+        for (int j = 0; j < n_kv; ++j) {
+            const int stage = j % kVStages;
+            if (!wait_all(&sm.v_full[stage], (j / kVStages) & 1)) {
+                if (lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
                 break;
             }
-            tc_fence_after_sync();
-            // Pass 1: row max over the visible keys of this tile (S stays in tensor memory;
-            // reading it twice keeps the row's 128 scores out of the register file).
-            const int nvis = lim - j * kN + 1;  // keys of this tile the row may see
-            float mx = -INFINITY, mx1 = -INFINITY;
-            {
-                // all four loads in flight before one wait: tensor-memory reads are cheap,
-                // their round trips are not
-                uint32_t sa[4][32];
+            uint8_t *vt = sm.v[stage];
+            // Each thread owns chunks cid, cid + 64, ... (chunk c: half c / 1024, key row
+            // (c / 8) % 128) through both passes, so no other thread touches them.
+            // pass 1: keys at or past L hold anything (even NaN): zero those rows so their
+            // zero weights contribute exactly zero (zero has the same bits in bf16 and f16);
+            // find the largest magnitude (as bf16 bits) of the rest.
+            const int valid = L - j * kN;
+            uint32_t mx = 0u;
+            constexpr int kBatch = 8;  // chunks in flight per thread
+#pragma unroll 1
+            for (int c0 = cid; c0 < kChunks16; c0 += kBatch * kConvThreads) {
+                uint4 w[kBatch];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, sa[cc]);
-                tmem_wait_ld();
+                for (int i = 0; i < kBatch; ++i)
+                    w[i] = *reinterpret_cast<const uint4 *>(vt + 16 * (c0 + i * kConvThreads));
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    if (nvis >= 32 * cc + 32) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            mx = fmaxf(mx, __uint_as_float(sa[cc][e]));
-                            mx1 = fmaxf(mx1, __uint_as_float(sa[cc][e + 1]));
-                        }
+                for (int i = 0; i < kBatch; ++i) {
+                    const int c = c0 + i * kConvThreads;
+                    if (((c >> 3) & (kN - 1)) >= valid) {
+                        *reinterpret_cast<uint4 *>(vt + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
                     } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            mx = fmaxf(mx, (32 * cc + e < nvis) ? __uint_as_float(sa[cc][e]) : -INFINITY);
+                        mx = umax16x2(mx, umax16x2(umax16x2(w[i].x & 0x7fff7fffu, w[i].y & 0x7fff7fffu),
+                                                   umax16x2(w[i].z & 0x7fff7fffu, w[i].w & 0x7fff7fffu)));
                     }
                 }
             }
-            mx = fmaxf(mx, mx1);
-            mx *= c;  // c > 0: the max commutes with the scale
-            const bool need = mx > m_ref + kRescaleThreshold;
-            const float new_ref = need ? mx : m_ref;
-            const float mref0 = new_ref == -INFINITY ? 0.f : new_ref;
-            const float alpha = ex2_approx(m_ref - mref0);
-
-            if (j > 0 && __any_sync(kAll, need)) {
-                // O must not be touched while PV(j-1) still accumulates into it
-                if (!wait_all(&sm.pv_done[q], (j - 1) & 1)) {
-                    ok = false;
+            const bool big = (mx & 0xffffu) >= kF16Limit || (mx >> 16) >= kF16Limit;
+            // exchange the verdict with the other converter warp: (j + 1) * 2 + flag, and a
+            // bounded wait for the partner's entry of this tile
+            const int mine = ((j + 1) << 1) | (__any_sync(kAll, big) ? 1 : 0);
+            volatile int *xo = &sm.conv_ovf[stage][0];
+            if (lane == 0) xo[cw] = mine;
+            int theirs = xo[cw ^ 1];
+            if ((theirs >> 1) != j + 1) {
+                const unsigned long long t0 = global_timer_ns();
+                while ((theirs >> 1) != j + 1 && global_timer_ns() - t0 < kWaitLimitNs) theirs = xo[cw ^ 1];
+            }
+            if (__any_sync(kAll, (theirs >> 1) != j + 1)) {
+                if (lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
+                break;
+            }
+            const bool keep_bf16 = ((mine | theirs) & 1) != 0;
+            if (!keep_bf16) {
+                // pass 2: bf16 -> f16 in place (bf16 -> fp32 is exact; fp32 -> f16 rounds
+                // to nearest, magnitudes under 2^-14 becoming f16 subnormals)
+#pragma unroll 1
+                for (int c0 = cid; c0 < kChunks16; c0 += kBatch * kConvThreads) {
+                    uint4 w[kBatch];
+#pragma unroll
+                    for (int i = 0; i < kBatch; ++i)
+                        w[i] = *reinterpret_cast<const uint4 *>(vt + 16 * (c0 + i * kConvThreads));
+#pragma unroll
+                    for (int i = 0; i < kBatch; ++i) {
+                        w[i].x = pack_f16(__uint_as_float(w[i].x << 16), __uint_as_float(w[i].x & 0xffff0000u));
+                        w[i].y = pack_f16(__uint_as_float(w[i].y << 16), __uint_as_float(w[i].y & 0xffff0000u));
+                        w[i].z = pack_f16(__uint_as_float(w[i].z << 16), __uint_as_float(w[i].z & 0xffff0000u));
+                        w[i].w = pack_f16(__uint_as_float(w[i].w << 16), __uint_as_float(w[i].w & 0xffff0000u));
+                        *reinterpret_cast<uint4 *>(vt + 16 * (c0 + i * kConvThreads)) = w[i];
+                    }
+                }
+            }
+            // the tensor core (async proxy) reads what these generic stores wrote
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (cw == 0) sm.v_bf16[stage] = keep_bf16 ? 1 : 0;
+                mbar_arrive(&sm.v_ready[stage]);
+            }
+            // stage of tile j - 1 -> tile j + kVStages - 1, once PV(j - 1) has read it
+            if (cw == 0 && j >= 1 && j + kVStages - 1 < n_kv) {
+                if (!wait_all(&sm.v_empty[(j - 1) % kVStages], ((j - 1) / kVStages) & 1)) {
+                    if (lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
                     break;
                 }
-                tc_fence_after_sync();
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + 32 * cc, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(tO + 32 * cc, o);
-                }
+                load_v(j + kVStages - 1);
             }
-            // Pass 2: P = 2^(s*c - ref) (0 past the visible keys), written over S in
-            // tensor memory chunk by chunk: the 32 keys of chunk cc (columns [32cc, 32cc+32)
-            // of S) become 16 columns of bf16 value pairs then 16 of bf16 residual pairs in
-            // those same columns, so a store never lands on scores not yet read.  Keys go
-            // in pairs through the paired fp32 instructions.
-            const unsigned long long c2 = f2_pack(c, c), nref2 = f2_pack(-mref0, -mref0);
-            const unsigned long long neg1 = f2_pack(-1.f, -1.f);
-            unsigned long long sum2 = 0ull;  // (0.f, 0.f)
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t sr[32];
-                tmem_ld32(tS + 32 * cc, sr);
-                tmem_wait_ld();
-                if (nvis < 32 * cc + 32) {  // diagonal / tail tile: scores past nvis -> -inf
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * cc + e >= nvis) sr[e] = __float_as_uint(-INFINITY);
-                }
-                uint32_t hi[16], lo[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
-                                     c2, nref2), x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    const unsigned long long pp = f2_pack(p0, p1);
-                    sum2 = f2_add(sum2, pp);
-                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    hi[e] = *reinterpret_cast<uint32_t *>(&h);
-                    const unsigned long long hf = f2_pack(__uint_as_float(hi[e] << 16),
-                                                          __uint_as_float(hi[e] & 0xffff0000u));
-                    float r0, r1;
-                    f2_unpack(f2_fma(hf, neg1, pp), r0, r1);
-                    lo[e] = pack_bf16(r0, r1);
-                }
-                tmem_st16(tS + 32 * cc, hi);
-                tmem_st16(tS + 32 * cc + 16, lo);
-            }
-            float sum, sum_hi;
-            f2_unpack(sum2, sum, sum_hi);
-            sum += sum_hi;
-            tmem_wait_st();
-            l = l * alpha + sum;
-            m_ref = new_ref;
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full[q]);
         }
-        if (nk > 0 && ok && wait_all(&sm.pv_done[q], (nk - 1) & 1)) {
-            tc_fence_after_sync();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) +
-                                 ((size_t)(q0 + tok) * a.Hq + kvh * g + hh) * kD;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(tO + 32 * cc, o);
-                tmem_wait_ld();
-                if (valid_row) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(dst + 32 * cc + e) = w;
-                    }
+        // no copy may outlive the CTA
+        if (cw == 0 && lane == 0)
+            for (int j = max(0, issued_v - kVStages); j < issued_v; ++j)
+                if (!mbar_wait(&sm.v_full[j % kVStages], (j / kVStages) & 1)) {
+                    set_error(a.err, GQA_ERR_TIMEOUT);
+                    break;
                 }
-            }
-            if (valid_row && a.lse)
-                a.lse[(size_t)(q0 + tok) * a.Hq + kvh * g + hh] =
-                    l > 0.f ? (m_ref + __log2f(l)) * kLn2P : -INFINITY;
-        } else if (nk > 0 && lane == 0) {
-            set_error(a.err, GQA_ERR_TIMEOUT);
-        }
+    }
     }
 
     tc_fence_before_sync();

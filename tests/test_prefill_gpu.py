@@ -113,3 +113,25 @@ def test_chunked_prefill_full_config_sampled():
     rows, ref_o, ref_l = _sampled_prefill_oracle(case, 12)
     check(out[rows], lse[rows], ref_o, ref_l, "chunked prefill B=8 Lq=512")
     assert np.isfinite(out).all()
+
+
+def _scaled_v_case(scale_v, seed):
+    """The same chunked-prefill inputs with V multiplied by a power of two (exact in bf16)."""
+    case = inputs.make_prefill_case(3, 32, 8, 128, 16, [0, 300, 900], [77, 256, 160], seed=seed)
+    kv = case.kv
+    v = (kv.v_pages.float() * scale_v).to(torch.bfloat16)
+    kv2 = inputs.PagedKV(kv.k_pages, v, kv.page_table, kv.seq_lens, kv.page_size)
+    return case, inputs.PrefillCase(case.q, case.cu_q, kv2, case.Hq, case.Hk, case.head_dim,
+                                    case.scale, case.seed, case.max_q_len)
+
+
+@pytest.mark.parametrize("log2s", [-12, 12, 14, 20])
+def test_prefill_v_scale_covariance(log2s):
+    """O is linear in V: out(V 2^s) / 2^s must match the oracle on V.  2^-12 pushes most
+    values into the f16 subnormal range, 2^12 keeps them under 2^16, and 2^14 / 2^20 put
+    some (or all) V tiles beyond the f16 range, where the kernel keeps those tiles bf16."""
+    s = 2.0 ** log2s
+    base, case = _scaled_v_case(s, seed=11 + log2s)
+    ref_o, ref_l = oracle_prefill(base)
+    out, lse = run_prefill(case)
+    check(out / s, lse, ref_o, ref_l, f"V x 2^{log2s}")
