@@ -38,6 +38,7 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLazyRef = 8.0f;  // log2 units a score may pass the reference by
 
 // Ring sizes: the split kernel runs 3 CTAs per SM with a 64 KB ring; the balanced
 // kernel runs 2 per SM (more registers per thread) with a 96 KB ring.
@@ -110,8 +111,9 @@ struct WarpAttn {
     static constexpr int MT = TT / 16;  // 16-token halves of a tile
     uint32_t qf[NT][KT][2];
     float qmul;  // fp8 path: power-of-two prescale bringing q into f16 range
+    float vref;  // fp8 path: o holds O / vref (tile V scales enter P as vsc / vref)
     float o[NT][KT][4];
-    float m[NT][2], l[NT][2];
+    float m[NT][2], l[NT][2];  // reference (log2 units) and running sum per head column
 
     __device__ __forceinline__ static int dim0(int dt, int gq) {
         return FP8 ? dt * 16 + 4 * (gq >> 1) + (gq & 1) : dt * 16 + gq;
@@ -130,6 +132,7 @@ struct WarpAttn {
             m[nt][0] = m[nt][1] = -INFINITY;
             l[nt][0] = l[nt][1] = 0.f;
         }
+        vref = 0.f;
     }
 
     // q rows of the nh packed heads start at q_rows (row stride D).
@@ -246,61 +249,94 @@ struct WarpAttn {
             }
         }
 
-        // ---- online softmax (exp2 domain) over the tile, per packed head column
+        // ---- online softmax (exp2 domain) over the tile, per packed head column, with a
+        // lazily moved reference: m only moves when a score passes it by more than 2^8
+        // (so P <= 2^8), which needs the column max (3 shuffles) and an O rescale only on
+        // those rare tiles; every other tile is one vote.
         const float kmul = FP8 ? scale_log2 * ksc / qmul : scale_log2;
+        float x[MT][NT][4];
+        bool need = false;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                x[mt][nt][0] = (16 * mt + gq < valid) ? s[mt][nt][0] * kmul : -INFINITY;
+                x[mt][nt][1] = (16 * mt + gq < valid) ? s[mt][nt][1] * kmul : -INFINITY;
+                x[mt][nt][2] = (16 * mt + gq + 8 < valid) ? s[mt][nt][2] * kmul : -INFINITY;
+                x[mt][nt][3] = (16 * mt + gq + 8 < valid) ? s[mt][nt][3] * kmul : -INFINITY;
+                need |= fmaxf(x[mt][nt][0], x[mt][nt][2]) > m[nt][0] + kLazyRef;
+                need |= fmaxf(x[mt][nt][1], x[mt][nt][3]) > m[nt][1] + kLazyRef;
+            }
+        if (__any_sync(kFull, need)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float alpha[2];
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(x[mt][nt][jj], x[mt][nt][jj + 2]));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+                    const float mnew = fmaxf(m[nt][jj], mx);
+                    alpha[jj] = fast_exp2(m[nt][jj] - (mnew == -INFINITY ? 0.f : mnew));
+                    l[nt][jj] *= alpha[jj];
+                    m[nt][jj] = mnew;
+                }
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt) {
+                    o[nt][dt][0] *= alpha[0];
+                    o[nt][dt][1] *= alpha[1];
+                    o[nt][dt][2] *= alpha[0];
+                    o[nt][dt][3] *= alpha[1];
+                }
+            }
+        }
+        // fp8: P enters the P.V product as P * vsc / vref, so the MMAs accumulate straight
+        // into o; vref follows the V scale when the ratio leaves [2^-8, 2^7] (keeping the
+        // f16 P under 2^15) and stays put for an all-zero page (vsc = 0).
+        float f = 1.f;
+        if (FP8) {
+            if (vref == 0.f) vref = vsc > 0.f ? vsc : 1.f;
+            f = vsc / vref;
+            if (f > 128.f || (f > 0.f && f < 1.f / 256.f)) {
+                const float r = vref / vsc;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int dt = 0; dt < KT; ++dt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[nt][dt][e] *= r;
+                vref = vsc;
+                f = 1.f;
+            }
+        }
         uint32_t pb[MT][NT][2], pbl[MT][NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float p[MT][4], alpha[2];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                float x[MT][2];
-                float mx = -INFINITY;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    x[mt][0] = (16 * mt + gq < valid) ? s[mt][nt][jj] * kmul : -INFINITY;
-                    x[mt][1] = (16 * mt + gq + 8 < valid) ? s[mt][nt][jj + 2] * kmul : -INFINITY;
-                    mx = fmaxf(mx, fmaxf(x[mt][0], x[mt][1]));
-                }
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                const float mnew = fmaxf(m[nt][jj], mx);
-                const float mref = mnew == -INFINITY ? 0.f : mnew;
-                alpha[jj] = fast_exp2(m[nt][jj] - mref);
-                float sum = 0.f;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    p[mt][jj] = fast_exp2(x[mt][0] - mref);
-                    p[mt][jj + 2] = fast_exp2(x[mt][1] - mref);
-                    sum += p[mt][jj] + p[mt][jj + 2];
-                }
-                l[nt][jj] = l[nt][jj] * alpha[jj] + sum;
-                m[nt][jj] = mnew;
-            }
+            const float mr0 = m[nt][0] == -INFINITY ? 0.f : m[nt][0];
+            const float mr1 = m[nt][1] == -INFINITY ? 0.f : m[nt][1];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
+                const float p0 = fast_exp2(x[mt][nt][0] - mr0), p1 = fast_exp2(x[mt][nt][1] - mr1);
+                const float p2 = fast_exp2(x[mt][nt][2] - mr0), p3 = fast_exp2(x[mt][nt][3] - mr1);
+                l[nt][0] += p0 + p2;
+                l[nt][1] += p1 + p3;
                 if (!FP8) {
                     // P as a bf16 value plus its bf16 residual: O += V^T P_hi^T + V^T P_lo^T
                     // keeps the weights at ~16 bits (one bf16 P costs up to 2^-9 per weight).
                     uint32_t h0, l0, h1, l1;
-                    split_bf16x2(p[mt][0], p[mt][1], h0, l0);
-                    split_bf16x2(p[mt][2], p[mt][3], h1, l1);
+                    split_bf16x2(p0, p1, h0, l0);
+                    split_bf16x2(p2, p3, h1, l1);
                     pb[mt][nt][0] = movmatrix_trans(h0);
                     pb[mt][nt][1] = movmatrix_trans(h1);
                     pbl[mt][nt][0] = movmatrix_trans(l0);
                     pbl[mt][nt][1] = movmatrix_trans(l1);
                 } else {
-                    pb[mt][nt][0] = movmatrix_trans(pack_f16(p[mt][0], p[mt][1]));
-                    pb[mt][nt][1] = movmatrix_trans(pack_f16(p[mt][2], p[mt][3]));
+                    pb[mt][nt][0] = movmatrix_trans(pack_f16(p0 * f, p1 * f));
+                    pb[mt][nt][1] = movmatrix_trans(pack_f16(p2 * f, p3 * f));
                 }
-            }
-#pragma unroll
-            for (int dt = 0; dt < KT; ++dt) {
-                o[nt][dt][0] *= alpha[0];
-                o[nt][dt][1] *= alpha[1];
-                o[nt][dt][2] *= alpha[0];
-                o[nt][dt][3] *= alpha[1];
             }
         }
 
@@ -325,12 +361,6 @@ struct WarpAttn {
             // fp8 V: plain ldmatrix gives each lane 4 consecutive dims of one token;
             // after conversion, movmatrix transposes 8x8 blocks into the A layout (dims
             // permuted within each 16-dim tile; dim0/dim1 undo it when O is written).
-            // The tile's P.V is summed apart and scaled once by the tile's V scale.
-            float pv[NT][KT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int dt = 0; dt < KT; ++dt) pv[nt][dt][0] = pv[nt][dt][1] = pv[nt][dt][2] = pv[nt][dt][3] = 0.f;
             const int j = lane >> 3;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
@@ -347,21 +377,23 @@ struct WarpAttn {
                                           movmatrix_trans(e4m3x2_to_f16x2(hi_t & 0xffff)),
                                           movmatrix_trans(e4m3x2_to_f16x2(hi_t >> 16))};
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) mma_f16(pv[nt][2 * qd + h], af, pb[mt][nt][0], pb[mt][nt][1]);
+                        for (int nt = 0; nt < NT; ++nt) mma_f16(o[nt][2 * qd + h], af, pb[mt][nt][0], pb[mt][nt][1]);
                     }
                 }
             }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int dt = 0; dt < KT; ++dt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) o[nt][dt][e] += vsc * pv[nt][dt][e];
         }
     }
 
     // Sum the per-lane partial sums l over the 8 lanes sharing a head column.
     __device__ __forceinline__ void finish_l() {
+        if (FP8 && vref != 0.f) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[nt][dt][e] *= vref;
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
