@@ -619,6 +619,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 // merging pieces) never holds up the other warps' streams.
 
 constexpr int kMinTilesPerWorker = 16;
+// A launch whose units average more than this many workers each merges pieces up a
+// tree (the TREE instance); otherwise the last piece of a unit merges all of them.  The
+// two are separate instances so that neither merge's registers burden the other's loop.
+constexpr int kTreeMinWorkersPerUnit = 24;
 
 __device__ __forceinline__ long long sk_start(long long W, long long T, long long NW) {
     return W >= NW ? T : (W * T) / NW;
@@ -662,8 +666,7 @@ __device__ __forceinline__ void flat_next(FlatPos &p, const int *pre, int U) {
 // Merge of every piece of one unit (pieces of workers wfirst..wlast; side 1 for the
 // first, side 0 for the rest) by one online log-sum-exp pass.  Lane owns dims
 // [DV*lane, DV*lane + DV) of every head; each piece's loads are independent of each
-// other.  Kept out of line: it runs once per shared unit and its arrays would otherwise
-// crowd the streaming loop's registers.
+// other.
 template <int D, int HW>
 __device__ __forceinline__ void merge_pieces(const float *pieces, long long wfirst, long long wlast,
                                           int slot_floats, int hpc, int nh, __nv_bfloat16 *out_rows,
@@ -715,7 +718,130 @@ __device__ __forceinline__ void merge_pieces(const float *pieces, long long wfir
     }
 }
 
-template <int D, int NT, bool FP8, int TT>
+// Merge tree for a unit cut into pieces (TREE instance; see the consumer loop):
+// this warp owns leaf `leaf` with its finished state in st; it writes its piece, then
+// climbs while it is the second child to arrive, and the warp reaching the root writes
+// the unit's output.
+template <int D, int NT, bool FP8, int TT, int HW>
+__device__ __forceinline__ void merge_tree(WarpAttn<D, NT, FP8, TT> &st, const DecodeArgs &a,
+                                           long long wfirst, int np, int leaf, int slot_floats,
+                                           int heads_per_cta, int nh, size_t row0, int lane) {
+    using WA = WarpAttn<D, NT, FP8, TT>;
+    constexpr int KT = D / 16;
+    const int gq = lane >> 2, cq = lane & 3;
+    auto slot_of = [&](int leaf) -> float * {
+        return a.pieces + (size_t)((wfirst + leaf) * 2 + (leaf == 0 ? 1 : 0)) * slot_floats;
+    };
+    // own result, normalised, LSE in log2 units
+    float lse2[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const float l = st.l[nt][jj];
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            lse2[nt][jj] = l > 0.f ? st.m[nt][jj] + __log2f(l) : -INFINITY;
+#pragma unroll
+            for (int dt = 0; dt < KT; ++dt) {
+                st.o[nt][dt][jj] *= inv;
+                st.o[nt][dt][jj + 2] *= inv;
+            }
+        }
+    auto publish = [&](float *slot) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int h = nt * 8 + 2 * cq + jj;
+                if (h >= nh) continue;
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt) {
+                    __stcg(slot + h * D + WA::dim0(dt, gq), st.o[nt][dt][jj]);
+                    __stcg(slot + h * D + WA::dim1(dt, gq), st.o[nt][dt][jj + 2]);
+                }
+                if (gq == 0) __stcg(slot + heads_per_cta * D + h, lse2[nt][jj] * kLn2);
+            }
+        __threadfence();
+        __syncwarp();
+    };
+    // fold the piece at `so` into the registers: left = registers if reg_left
+    auto fold = [&](const float *so, bool reg_left) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int h = nt * 8 + 2 * cq + jj;
+                if (h >= nh) continue;
+                const float ls = __ldcg(so + heads_per_cta * D + h) * kLog2e;
+                const float lL = reg_left ? lse2[nt][jj] : ls, lR = reg_left ? ls : lse2[nt][jj];
+                const float M = fmaxf(lL, lR);
+                const float wL = lL == -INFINITY ? 0.f : fast_exp2(lL - M);
+                const float wR = lR == -INFINITY ? 0.f : fast_exp2(lR - M);
+                const float sum = wL + wR;
+                const float inv = sum > 0.f ? 1.f / sum : 0.f;
+                const float cL = wL * inv, cR = wR * inv;
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt) {
+                    const float s0 = __ldcg(so + h * D + WA::dim0(dt, gq));
+                    const float s1 = __ldcg(so + h * D + WA::dim1(dt, gq));
+                    const float o0 = st.o[nt][dt][jj], o1 = st.o[nt][dt][jj + 2];
+                    const float L0 = reg_left ? o0 : s0, R0 = reg_left ? s0 : o0;
+                    const float L1 = reg_left ? o1 : s1, R1 = reg_left ? s1 : o1;
+                    st.o[nt][dt][jj] = cR == 0.f ? cL * L0 : fmaf(cR, R0, cL * L0);
+                    st.o[nt][dt][jj + 2] = cR == 0.f ? cL * L1 : fmaf(cR, R1, cL * L1);
+                }
+                lse2[nt][jj] = sum > 0.f ? M + __log2f(sum) : -INFINITY;
+            }
+    };
+    int levels = 0;
+    while ((1 << levels) < np) ++levels;
+    int node = leaf, lv = 0;
+    bool mine = true;  // this warp writes the unit's output
+    publish(slot_of(node));
+    while (lv < levels) {
+        const int sib = node ^ 1;
+        if ((sib << lv) >= np) {  // no sibling: the node's result is its parent's
+            node >>= 1;
+            ++lv;
+            continue;
+        }
+        const int p0 = (node >> 1) << (lv + 1);  // parent's leftmost leaf
+        int *ctr = a.counters + ((size_t)((wfirst + p0) * 2 + (p0 == 0 ? 1 : 0)) * kTreeLevels + lv + 1);
+        int second = 0;
+        if (lane == 0) {
+            second = atomicAdd(ctr, 1) == 1;
+            if (second) *ctr = 0;  // ready for the next launch
+        }
+        if (!__shfl_sync(kFull, second, 0)) {
+            mine = false;
+            break;
+        }
+        __threadfence();
+        fold(slot_of(sib << lv), node < sib);
+        node >>= 1;
+        ++lv;
+        if (lv < levels) publish(slot_of(node << lv));
+    }
+    if (mine) {
+        // the root: the unit's output
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int h = nt * 8 + 2 * cq + jj;
+                if (h >= nh) continue;
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) + (row0 + h) * D;
+#pragma unroll
+                for (int dt = 0; dt < KT; ++dt) {
+                    dst[WA::dim0(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj]);
+                    dst[WA::dim1(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj + 2]);
+                }
+                if (gq == 0 && a.lse) a.lse[row0 + h] = lse2[nt][jj] * kLn2;
+            }
+    }
+}
+
+template <int D, int NT, bool FP8, int TT, bool TREE>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     decode_sk_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const DecodeArgs a,
@@ -908,37 +1034,51 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
                                               : -INFINITY;
                 }
         } else {
-            // a piece of a unit shared with neighbouring workers: side 0 = the unit began
+            // A piece of a unit shared with neighbouring workers: side 0 = the unit began
             // before this worker's range, side 1 = it begins here and continues after.
-            const int side = us < s_w ? 0 : 1;
-            float *slot = a.pieces + (size_t)(Wme * 2 + side) * slot_floats;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int h = nt * 8 + 2 * cq + jj;
-                    if (h >= nh) continue;
-                    const float inv = 1.f / st.l[nt][jj];
-#pragma unroll
-                    for (int dt = 0; dt < KT; ++dt) {
-                        slot[h * D + WA::dim0(dt, gq)] = st.o[nt][dt][jj] * inv;
-                        slot[h * D + WA::dim1(dt, gq)] = st.o[nt][dt][jj + 2] * inv;
-                    }
-                    if (gq == 0) slot[heads_per_cta * D + h] = (st.m[nt][jj] + __log2f(st.l[nt][jj])) * kLn2;
-                }
-            __threadfence();
-            __syncwarp();
+            // Each piece (leaf k = worker wfirst + k) is written normalised with its LSE
+            // (natural log).  Launches whose units span few workers: the last piece to
+            // finish merges all of them in one pass.  Launches whose units span many
+            // (TREE): the pieces are merged up a binary tree: at level lv, node
+            // n covers leaves [n 2^lv, (n+1) 2^lv); of the two children of a node, the one
+            // whose result is ready second merges the other's (loaded from the slot of its
+            // leftmost leaf) with its own (in registers), left operand first, so the result
+            // does not depend on the order in which workers finish.
             const long long wfirst = sk_worker_of(us, T, NW), wlast = sk_worker_of(ue - 1, T, NW);
-            const int npieces = (int)(wlast - wfirst + 1);
-            int last = 0;
-            if (lane == 0) last = atomicAdd(a.counters + (size_t)b * U + y, 1) == npieces - 1;
-            last = __shfl_sync(kFull, last, 0);
-            if (last) {
+            const int np = (int)(wlast - wfirst + 1);
+            if (!TREE) {
+                const int side = us < s_w ? 0 : 1;
+                float *slot = a.pieces + (size_t)(Wme * 2 + side) * slot_floats;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int h = nt * 8 + 2 * cq + jj;
+                        if (h >= nh) continue;
+                        const float inv = 1.f / st.l[nt][jj];
+#pragma unroll
+                        for (int dt = 0; dt < KT; ++dt) {
+                            slot[h * D + WA::dim0(dt, gq)] = st.o[nt][dt][jj] * inv;
+                            slot[h * D + WA::dim1(dt, gq)] = st.o[nt][dt][jj + 2] * inv;
+                        }
+                        if (gq == 0) slot[heads_per_cta * D + h] = (st.m[nt][jj] + __log2f(st.l[nt][jj])) * kLn2;
+                    }
                 __threadfence();
-                merge_pieces<D, HW>(a.pieces, wfirst, wlast, slot_floats, heads_per_cta, nh,
-                                    reinterpret_cast<__nv_bfloat16 *>(a.out) + row0 * D,
-                                    a.lse ? a.lse + row0 : nullptr, lane);
-                if (lane == 0) a.counters[(size_t)b * U + y] = 0;  // ready for the next launch
+                __syncwarp();
+                int *ctr = a.counters + kTreeCounters + (size_t)b * U + y;
+                int last = 0;
+                if (lane == 0) last = atomicAdd(ctr, 1) == np - 1;
+                last = __shfl_sync(kFull, last, 0);
+                if (last) {
+                    __threadfence();
+                    merge_pieces<D, HW>(a.pieces, wfirst, wlast, slot_floats, heads_per_cta, nh,
+                                        reinterpret_cast<__nv_bfloat16 *>(a.out) + row0 * D,
+                                        a.lse ? a.lse + row0 : nullptr, lane);
+                    if (lane == 0) *ctr = 0;  // ready for the next launch
+                }
+            } else {
+                merge_tree<D, NT, FP8, TT, HW>(st, a, wfirst, np, (int)(Wme - wfirst), slot_floats,
+                                               heads_per_cta, nh, row0, lane);
             }
         }
         st.reset();
@@ -959,10 +1099,12 @@ cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtenso
     if (a.stream_k) {
         const size_t smem =
             sizeof(Smem<D, FP8, kRingBalanced, TT>) + 1024 + sizeof(int) * (size_t)(a.B + 1);
-        cudaError_t e = cudaFuncSetAttribute(decode_sk_kernel<D, NT, FP8, TT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const long long units = (long long)a.B * a.Hk * chunks;
+        const bool tree = (long long)a.grid * kConsumerWarps > kTreeMinWorkersPerUnit * units;
+        auto kern = tree ? decode_sk_kernel<D, NT, FP8, TT, true> : decode_sk_kernel<D, NT, FP8, TT, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_sk_kernel<D, NT, FP8, TT><<<a.grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
+        kern<<<a.grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
         return cudaGetLastError();
     }
     const size_t smem = sizeof(Smem<D, FP8, kRingSplit, TT>) + 1024;

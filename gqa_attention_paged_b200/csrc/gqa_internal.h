@@ -28,7 +28,7 @@ struct DecodeArgs {
     int *err;
     // balanced persistent schedule (num_splits == 0, B <= kStreamMaxBatch)
     int stream_k;
-    int *counters;  // [B * units per sequence], zero between launches
+    int *counters;  // [2 * workers][kTreeLevels] tree, then [B * units] flat merge counters; zero between launches
     float *pieces;  // [workers * 2][heads per CTA][D + 1]
     int grid;       // persistent CTAs
 };
@@ -41,10 +41,17 @@ constexpr int kStreamCtasPerSm = 2;
 constexpr int kStreamMaxSms = 160;
 constexpr int kStreamWorkersPerCta = 4;
 
+// Levels of the balanced schedule's merge tree (pieces per unit <= workers < 2^11).
+constexpr int kTreeLevels = 12;
+constexpr int kStreamMaxWorkers = kStreamMaxSms * kStreamCtasPerSm * kStreamWorkersPerCta;
+
 // Bytes at the start of a decode workspace that must be zero before a launch: the error
-// word header and, for the balanced schedule, one merge counter per (sequence, head).
+// word header, then the balanced schedule's merge counters: one per (piece slot, tree
+// level) for 2 slots per worker of the largest grid, then one per (sequence, head) for
+// units merged by their last piece.
+constexpr size_t kTreeCounters = (size_t)2 * kStreamMaxWorkers * kTreeLevels;
 inline size_t decode_zero_prefix_bytes(int B, int Hq) {
-    return kWorkspaceHeader + ((size_t)B * Hq * sizeof(int) + 255) / 256 * 256;
+    return kWorkspaceHeader + ((kTreeCounters + (size_t)B * Hq) * sizeof(int) + 255) / 256 * 256;
 }
 
 // Launch the decode kernel (and nothing else) on `stream`.  The tensor maps describe the

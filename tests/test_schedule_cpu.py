@@ -4,7 +4,8 @@ share.  The formulas are the ones decode_sk_kernel evaluates (restated here): wo
 owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // 16)); the owner
 of tile t is ((t+1)*NW + T-1)//T - 1;
 a unit cut between workers leaves one piece per worker, side 1 for the worker where the
-unit begins and side 0 for the others, and the last of them merges all pieces."""
+unit begins and side 0 for the others; the pieces are merged up a binary tree whose
+internal nodes are claimed by the second of their two children to arrive."""
 import itertools
 import random
 
@@ -109,3 +110,68 @@ def test_slot_indices_stay_in_the_workspace():
         U = Hk * ((g + hpc - 1) // hpc)
         assert B * U <= B * Hq
         assert 2 * (workers - 1) + 1 < 2 * workers
+
+
+def tree_merge(np_, order, levels_cap=12):
+    """Replay the merge-tree protocol for np_ pieces whose leaf owners finish in `order`.
+    Each owner climbs: no sibling -> move up; else arrive at the parent's counter; the
+    first arrival stops, the second merges (left operand first) and climbs on.  Returns
+    the root's operand tree and the counter ids used."""
+    levels = 0
+    while (1 << levels) < np_:
+        levels += 1
+    assert levels < levels_cap
+    counters, results, roots, used = {}, {k: k for k in range(np_)}, [], set()
+    pending = {}
+    for k in order:
+        node, lv, val = k, 0, k
+        while lv < levels:
+            sib = node ^ 1
+            if (sib << lv) >= np_:
+                node >>= 1
+                lv += 1
+                continue
+            p0 = (node >> 1) << (lv + 1)
+            cid = (p0, lv + 1)
+            used.add(cid)
+            counters[cid] = counters.get(cid, 0) + 1
+            if counters[cid] == 1:
+                pending[(lv, node)] = val
+                break
+            other = pending.pop((lv, sib))
+            val = (val, other) if node < sib else (other, val)
+            node >>= 1
+            lv += 1
+        else:
+            roots.append(val)
+    return roots, counters, used
+
+
+def _tree_of(np_):
+    levels = 0
+    while (1 << levels) < np_:
+        levels += 1
+    def build(lv, node):
+        lo = node << lv
+        if lo >= np_:
+            return None
+        if lv == 0:
+            return lo
+        l, r = build(lv - 1, 2 * node), build(lv - 1, 2 * node + 1)
+        return l if r is None else (l, r)
+    return build(levels, 0)
+
+
+@pytest.mark.parametrize("np_", [2, 3, 4, 5, 7, 8, 9, 16, 37, 100, 1280])
+def test_merge_tree_has_one_root_and_a_fixed_shape(np_):
+    rng = random.Random(np_)
+    want = _tree_of(np_)
+    for trial in range(20):
+        order = list(range(np_))
+        rng.shuffle(order)
+        roots, counters, used = tree_merge(np_, order)
+        assert len(roots) == 1, "exactly one worker writes the unit"
+        assert roots[0] == want, "the result must not depend on the arrival order"
+        assert all(c == 2 for c in counters.values()), "every counter is claimed by two children"
+        # counter ids stay inside [2 * workers][12]: leaf slot < 2 * 1280, level < 12
+        assert all(p0 < 1280 and 1 <= lv < 12 for p0, lv in used)
