@@ -759,7 +759,7 @@ __device__ __forceinline__ void merge_tree(WarpAttn<D, NT, FP8, TT> &st, const D
                     __stcg(slot + h * D + WA::dim0(dt, gq), st.o[nt][dt][jj]);
                     __stcg(slot + h * D + WA::dim1(dt, gq), st.o[nt][dt][jj + 2]);
                 }
-                if (gq == 0) __stcg(slot + heads_per_cta * D + h, lse2[nt][jj] * kLn2);
+                if (gq == 0) __stcg(slot + heads_per_cta * D + h, lse2[nt][jj]);
             }
         __threadfence();
         __syncwarp();
@@ -772,7 +772,7 @@ __device__ __forceinline__ void merge_tree(WarpAttn<D, NT, FP8, TT> &st, const D
             for (int jj = 0; jj < 2; ++jj) {
                 const int h = nt * 8 + 2 * cq + jj;
                 if (h >= nh) continue;
-                const float ls = __ldcg(so + heads_per_cta * D + h) * kLog2e;
+                const float ls = __ldcg(so + heads_per_cta * D + h);
                 const float lL = reg_left ? lse2[nt][jj] : ls, lR = reg_left ? ls : lse2[nt][jj];
                 const float M = fmaxf(lL, lR);
                 const float wL = lL == -INFINITY ? 0.f : fast_exp2(lL - M);
@@ -1037,7 +1037,9 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
             // A piece of a unit shared with neighbouring workers: side 0 = the unit began
             // before this worker's range, side 1 = it begins here and continues after.
             // Each piece (leaf k = worker wfirst + k) is written normalised with its LSE
-            // (natural log).  Launches whose units span few workers: the last piece to
+            // (natural log for the flat merge, log2 units in the tree, where a value must not
+            // depend on whether it came through a slot).  Launches whose units span few
+            // workers: the last piece to
             // finish merges all of them in one pass.  Launches whose units span many
             // (TREE): the pieces are merged up a binary tree: at level lv, node
             // n covers leaves [n 2^lv, (n+1) 2^lv); of the two children of a node, the one
