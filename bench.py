@@ -288,7 +288,8 @@ def run_prefill_bench(a):
         "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(tf / peak, 4), "traffic": None,
                      "peak_source": f"{kind} (bf16_tflops, burst cuBLAS GEMM)"},
-        "gpu_launches": a.steps, "clocks": clk}))
+        "gpu_launches": 2 * a.steps,  # the plan kernel and the prefill kernel per step
+        "clocks": clk}))
     return 0
 
 

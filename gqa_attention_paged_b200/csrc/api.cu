@@ -153,10 +153,9 @@ size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int 
 }
 
 size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim) {
-    (void)total_q;
     (void)Hq;
     (void)head_dim;
-    return kWorkspaceHeader;
+    return prefill_workspace_bytes(total_q < 0 ? 0 : total_q);
 }
 
 int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
@@ -260,6 +259,9 @@ int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
     if (B == 0 || total_q == 0 || max_q_len == 0) return GQA_OK;
     const int g = Hq / Hk;
     const int T = 128 / g;
+    // work items (pairs of query tiles) per sequence, and the launch's upper bound on them
+    const int64_t items_per_seq = ((int64_t)max_q_len + 2 * T - 1) / (2 * T);
+    if (items_per_seq > 65535 || (int64_t)B * items_per_seq * Hk > INT32_MAX) return GQA_ERR_SHAPE;
     const int64_t rows = (int64_t)num_pages * Hk * page_size;
     CUtensorMap kmap, vmap, qmap;
     if (encode_kv_map(&kmap, k_pages, GQA_KV_BF16, head_dim, rows, 16) != GQA_OK ||
@@ -285,6 +287,7 @@ int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
     a.out = out;
     a.lse = lse;
     a.err = reinterpret_cast<int *>(workspace);
+    a.plan = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + kWorkspaceHeader);
     return launch_prefill(a, kmap, vmap, qmap, stream) == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
 }
 

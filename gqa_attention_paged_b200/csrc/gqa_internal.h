@@ -80,7 +80,17 @@ struct PrefillArgs {
     void *out;
     float *lse;
     int *err;
+    int *plan;  // [1 + items]: count, then (b << 16 | query-tile pair) longest first
 };
+
+// Work items of a prefill launch (pairs of query tiles) are ordered longest first by a
+// one-CTA plan kernel; costs are binned by KV tiles up to this many.
+constexpr int kPlanBins = 4096;
+// Bytes of the prefill workspace: the error-word header, then the plan (one int per
+// item, at most one item per query token, plus the count).
+inline size_t prefill_workspace_bytes(int total_q) {
+    return kWorkspaceHeader + ((size_t)(total_q + 1) * sizeof(int) + 255) / 256 * 256;
+}
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap,
                            const CUtensorMap &vmap, const CUtensorMap &qmap,

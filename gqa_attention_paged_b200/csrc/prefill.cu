@@ -5,7 +5,8 @@
 // prefill); its K/V are already the last Lq cached tokens, and query row i (position
 // L - Lq + i) attends to keys 0 .. L - Lq + i.
 //
-// One CTA = (two query tiles, kv head, sequence).  A tile packs the g query heads of the
+// One CTA = (two query tiles, kv head, sequence), launched longest first (a one-CTA plan
+// kernel orders the work items by the KV tiles they read, before each prefill launch).  A tile packs the g query heads of the
 // group with T = 128 / g tokens into 128 rows, row r = (token r / g, head r % g)
 // (PackGQA: "解锁GQA性能潜力：从批量大小敏感性到高效优化实践", PackGQA / NumSplits
 // section), so each K/V tile feeds every head of the group, twice (once per query tile).
@@ -273,6 +274,66 @@ __device__ __forceinline__ void softmax_role(PSmem &sm, const PrefillArgs &a, co
     }
 }
 
+// Longest-first order of the launch's work items.  Item (b, x) is query tiles 2x, 2x+1 of
+// sequence b; its cost is the number of 128-key tiles its later query tile reads.  One CTA
+// bins the items by cost (a counting sort), then writes them to plan[1..] from the highest
+// bin down, and the count to plan[0].  Items of equal cost keep no particular order:
+// each is computed on its own, so the outputs do not depend on it.
+__global__ void __launch_bounds__(1024)
+    prefill_plan_kernel(const PrefillArgs a, const int T, const int items_per_seq) {
+    __shared__ int hist[kPlanBins];
+    const int total = a.B * items_per_seq;
+    for (int i = threadIdx.x; i < kPlanBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    auto cost_of = [&](int idx, int &item) -> int {
+        const int b = idx / items_per_seq, x = idx % items_per_seq;
+        const int Lq = a.cu_q[b + 1] - a.cu_q[b];
+        if (x * 2 * T >= Lq) return -1;
+        const int L = a.seq_lens[b];
+        const int last = a.causal ? L - Lq + min(Lq, (x + 1) * 2 * T) - 1 : L - 1;
+        item = (b << 16) | x;
+        return min(max(last, 0) / kN + 1, kPlanBins - 1);
+    };
+    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+        int item;
+        const int c = cost_of(idx, item);
+        if (c >= 0) atomicAdd(&hist[c], 1);
+        if (idx % items_per_seq == 0) {
+            const int b = idx / items_per_seq;
+            if (a.cu_q[b + 1] - a.cu_q[b] > items_per_seq * 2 * T)
+                set_error(a.err, GQA_ERR_SHAPE);  // max_q_len below a chunk length
+        }
+    }
+    __syncthreads();
+    // exclusive offsets in descending cost order (warp 0; lane i owns a run of bins)
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        constexpr int per = kPlanBins / 32;
+        int sum = 0;
+        for (int i = 0; i < per; ++i) sum += hist[kPlanBins - 1 - (lane * per + i)];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(kAll, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int c = kPlanBins - 1 - (lane * per + i);
+            const int h = hist[c];
+            hist[c] = run;
+            run += h;
+        }
+        if (lane == 31) a.plan[0] = incl;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+        int item;
+        const int c = cost_of(idx, item);
+        if (c >= 0) a.plan[1 + atomicAdd(&hist[c], 1)] = item;
+    }
+}
+
 __global__ void __launch_bounds__(kThreadsP, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                    const __grid_constant__ CUtensorMap qmap, const PrefillArgs a, const int T) {
@@ -280,14 +341,17 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     PSmem &sm = *reinterpret_cast<PSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.z, kvh = blockIdx.y;
-    const int ct = gridDim.x - 1 - blockIdx.x;  // longest (latest) tiles first
+    // block i = (work item i / Hk in the plan's longest-first order, kv head i % Hk), so
+    // the longest items are dispatched first, all heads of an item together
+    const int kvh = blockIdx.x % a.Hk;
+    const int rank = blockIdx.x / a.Hk;
+    if (rank >= a.plan[0]) return;  // uniform for the whole CTA
+    const int item = a.plan[1 + rank];
+    const int b = item >> 16, ct = item & 0xffff;
     const int g = a.Hq / a.Hk;
     const int q0 = a.cu_q[b];
     const int Lq = a.cu_q[b + 1] - q0;
     const int i0 = ct * kQT * T;  // first token of query tile 0
-    if (blockIdx.x == 0 && threadIdx.x == 0 && Lq > (int)gridDim.x * kQT * T)
-        set_error(a.err, GQA_ERR_SHAPE);  // max_q_len below a chunk length
     if (i0 >= Lq) return;  // uniform for the whole CTA
     const int L = a.seq_lens[b];
     const int P = a.P;
@@ -602,10 +666,11 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap, const 
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int tiles = (a.max_q_len + kQT * T - 1) / (kQT * T);
-    if (tiles == 0 || a.B == 0) return cudaSuccess;
-    dim3 grid(tiles, a.Hk, a.B);
-    prefill_kernel<<<grid, kThreadsP, smem, stream>>>(kmap, vmap, qmap, a, T);
+    const int items_per_seq = (a.max_q_len + kQT * T - 1) / (kQT * T);
+    if (items_per_seq == 0 || a.B == 0) return cudaSuccess;
+    prefill_plan_kernel<<<1, 1024, 0, stream>>>(a, T, items_per_seq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    prefill_kernel<<<a.B * items_per_seq * a.Hk, kThreadsP, smem, stream>>>(kmap, vmap, qmap, a, T);
     return cudaGetLastError();
 }
 

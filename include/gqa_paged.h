@@ -179,7 +179,10 @@ int gqa_paged_decode_static_scratch(const void *q, const void *k_pages, const vo
                                     cudaStream_t stream);
 
 /*
- * Bytes of workspace gqa_paged_prefill() needs (the 256-byte error-word header).
+ * Bytes of workspace gqa_paged_prefill() needs for total_q query tokens: the 256-byte
+ * error-word header, then the launch plan (the count and one int per work item, a work
+ * item being two query tiles of one sequence: at most one per query token), rounded up to
+ * 256 bytes.  Hq and head_dim are accepted for symmetry with the decode call.
  */
 size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim);
 

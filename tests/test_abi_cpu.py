@@ -91,6 +91,8 @@ def test_host_helpers():
     assert lib.gqa_paged_gather(_fake(), _fake(), _fake(), 4, _fake(), _fake(), 2, 2, 64, 16, 8,
                                 3, _fake(), _fake(), None) == -2
     assert lib.gqa_get_error(None, None) == -1
+    for tq in (0, 1, 63, 64, 4096):
+        assert lib.gqa_paged_prefill_workspace_size(tq, 32, 128) == 256 + (4 * (tq + 1) + 255) // 256 * 256
 
 
 def test_binding_refuses_cpu_tensors():

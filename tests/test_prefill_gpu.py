@@ -75,7 +75,7 @@ def test_prefill_last_row_matches_gpu_decode():
 
 def test_prefill_max_q_len_too_small_sets_error():
     case = inputs.make_prefill_case(2, 8, 2, 128, 16, [10, 10], [40, 100], seed=6)
-    ws = binding.new_workspace(256, DEV)
+    ws = binding.new_workspace(binding.gqa_paged_prefill_workspace_size(140, 8, 128), DEV)
     run_prefill(case, max_q_len=40, workspace=ws)
     assert binding.gqa_get_error(ws) == -2
 
