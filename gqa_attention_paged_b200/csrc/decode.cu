@@ -76,8 +76,8 @@ struct alignas(1024) Smem {
     uint8_t tiles[C::kStages][2][C::kTileBytes];
     uint64_t full[C::kStages];
     uint64_t empty[C::kStages];
-    float kscale[C::kStages];
-    float vscale[C::kStages];
+    float kscale[C::kStages][2];  // per 16-token half of the tile
+    float vscale[C::kStages][2];
     TileRec rec[C::kStages];
     int abort_flag;
 };
@@ -190,8 +190,10 @@ struct WarpAttn {
     }
 
     // Fold one TT-token tile (valid tokens first, rows past them ignored) into the state.
+    // fp8: ksc[mt] / vsc[mt] are the K / V scales of the tile's 16-token half mt (two
+    // pages when a 32-token tile spans two 16-token pages).
     __device__ __forceinline__ void tile(uint8_t *kt, uint8_t *vt, int valid, float scale_log2,
-                                         float ksc, float vsc, int lane) {
+                                         const float (&ksc)[2], const float (&vsc)[2], int lane) {
         using C = Cfg<D, FP8, kRingSplit, TT>;
         const int gq = lane >> 2;
         if (valid < TT) {
@@ -253,17 +255,19 @@ struct WarpAttn {
         // lazily moved reference: m only moves when a score passes it by more than 2^8
         // (so P <= 2^8), which needs the column max (3 shuffles) and an O rescale only on
         // those rare tiles; every other tile is one vote.
-        const float kmul = FP8 ? scale_log2 * ksc / qmul : scale_log2;
+        float kmul[MT];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) kmul[mt] = FP8 ? scale_log2 * ksc[mt] / qmul : scale_log2;
         float x[MT][NT][4];
         bool need = false;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                x[mt][nt][0] = (16 * mt + gq < valid) ? s[mt][nt][0] * kmul : -INFINITY;
-                x[mt][nt][1] = (16 * mt + gq < valid) ? s[mt][nt][1] * kmul : -INFINITY;
-                x[mt][nt][2] = (16 * mt + gq + 8 < valid) ? s[mt][nt][2] * kmul : -INFINITY;
-                x[mt][nt][3] = (16 * mt + gq + 8 < valid) ? s[mt][nt][3] * kmul : -INFINITY;
+                x[mt][nt][0] = (16 * mt + gq < valid) ? s[mt][nt][0] * kmul[mt] : -INFINITY;
+                x[mt][nt][1] = (16 * mt + gq < valid) ? s[mt][nt][1] * kmul[mt] : -INFINITY;
+                x[mt][nt][2] = (16 * mt + gq + 8 < valid) ? s[mt][nt][2] * kmul[mt] : -INFINITY;
+                x[mt][nt][3] = (16 * mt + gq + 8 < valid) ? s[mt][nt][3] * kmul[mt] : -INFINITY;
                 need |= fmaxf(x[mt][nt][0], x[mt][nt][2]) > m[nt][0] + kLazyRef;
                 need |= fmaxf(x[mt][nt][1], x[mt][nt][3]) > m[nt][1] + kLazyRef;
             }
@@ -294,23 +298,27 @@ struct WarpAttn {
             }
         }
         // fp8: P enters the P.V product as P * vsc / vref, so the MMAs accumulate straight
-        // into o; vref follows the V scale when the ratio leaves [2^-8, 2^7] (keeping the
-        // f16 P under 2^15) and stays put for an all-zero page (vsc = 0).
-        float f = 1.f;
+        // into o; vref follows the tile's larger V scale when the ratio leaves [2^-8, 2^7]
+        // (keeping the f16 P under 2^15) and stays put for all-zero pages (vsc = 0).
+        float f[MT];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) f[mt] = 1.f;
         if (FP8) {
-            if (vref == 0.f) vref = vsc > 0.f ? vsc : 1.f;
-            f = vsc / vref;
-            if (f > 128.f || (f > 0.f && f < 1.f / 256.f)) {
-                const float r = vref / vsc;
+            const float vmax = MT == 2 ? fmaxf(vsc[0], vsc[1]) : vsc[0];
+            if (vref == 0.f) vref = vmax > 0.f ? vmax : 1.f;
+            const float fm = vmax / vref;
+            if (fm > 128.f || (fm > 0.f && fm < 1.f / 256.f)) {
+                const float r = vref / vmax;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int dt = 0; dt < KT; ++dt)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) o[nt][dt][e] *= r;
-                vref = vsc;
-                f = 1.f;
+                vref = vmax;
             }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) f[mt] = vsc[mt] / vref;
         }
         uint32_t pb[MT][NT][2], pbl[MT][NT][2];
 #pragma unroll
@@ -334,8 +342,8 @@ struct WarpAttn {
                     pbl[mt][nt][0] = movmatrix_trans(l0);
                     pbl[mt][nt][1] = movmatrix_trans(l1);
                 } else {
-                    pb[mt][nt][0] = movmatrix_trans(pack_f16(p0 * f, p1 * f));
-                    pb[mt][nt][1] = movmatrix_trans(pack_f16(p2 * f, p3 * f));
+                    pb[mt][nt][0] = movmatrix_trans(pack_f16(p0 * f[mt], p1 * f[mt]));
+                    pb[mt][nt][1] = movmatrix_trans(pack_f16(p2 * f[mt], p3 * f[mt]));
                 }
             }
         }
@@ -488,8 +496,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
                         issued = it + 1;
                     } else {
                         if (FP8) {
-                            sm.kscale[stage] = ks;
-                            sm.vscale[stage] = vs;
+                            sm.kscale[stage][0] = sm.kscale[stage][1] = ks;
+                            sm.vscale[stage][0] = sm.vscale[stage][1] = vs;
                         }
                         const int row = (ph * a.Hk + kvh) * P + (t0 + it * kTile) % P;
                         mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
@@ -534,8 +542,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
             fail = true;
             break;
         }
+        const float ksl[2] = {FP8 ? sm.kscale[stage][0] : 1.f, FP8 ? sm.kscale[stage][1] : 1.f};
+        const float vsl[2] = {FP8 ? sm.vscale[stage][0] : 1.f, FP8 ? sm.vscale[stage][1] : 1.f};
         st.tile(sm.tiles[stage][0], sm.tiles[stage][1], t1 - (t0 + it * kTile), scale_log2,
-                FP8 ? sm.kscale[stage] : 1.f, FP8 ? sm.vscale[stage] : 1.f, lane);
+                ksl, vsl, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[stage]);
     }
@@ -939,24 +949,50 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
             rec.tile = pos.tile;
             rec.valid = min(kTile, L - tok0);
             rec.f = s_w + r;
-            const int phys = __ldg(a.page_table + (size_t)pos.b * a.pt_stride + tok0 / P);
+            // a 32-token e4m3 tile on 16-token pages spans two pages: one box from each
+            const int32_t *ptb = a.page_table + (size_t)pos.b * a.pt_stride + tok0 / P;
+            const int phys = __ldg(ptb);
+            const bool two = kTile > P;
+            const bool second = two && tok0 + P < L;
+            const int phys2 = second ? __ldg(ptb + 1) : phys;
             sm.rec[stage] = rec;
-            if (phys < 0 || phys >= a.num_pages) {
+            if (phys < 0 || phys >= a.num_pages || phys2 < 0 || phys2 >= a.num_pages) {
                 set_error(a.err, GQA_ERR_BAD_PAGE);
                 mbar_arrive(&sm.full[stage]);  // no copy: the tile computes on stale data
             } else {
                 if (FP8) {
-                    sm.kscale[stage] = __ldg(a.k_scale + (size_t)phys * a.Hk + kvh);
-                    sm.vscale[stage] = __ldg(a.v_scale + (size_t)phys * a.Hk + kvh);
+                    sm.kscale[stage][0] = __ldg(a.k_scale + (size_t)phys * a.Hk + kvh);
+                    sm.vscale[stage][0] = __ldg(a.v_scale + (size_t)phys * a.Hk + kvh);
+                    sm.kscale[stage][1] = second ? __ldg(a.k_scale + (size_t)phys2 * a.Hk + kvh) : sm.kscale[stage][0];
+                    sm.vscale[stage][1] = second ? __ldg(a.v_scale + (size_t)phys2 * a.Hk + kvh) : sm.vscale[stage][0];
                 }
                 const int row = (phys * a.Hk + kvh) * P + tok0 % P;
-                mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
+                if (!two) {
+                    mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
 #pragma unroll
-                for (int bx = 0; bx < C::kBoxes; ++bx) {
-                    tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128, &kmap, &sm.full[stage],
-                                bx * C::kBoxCols, row, pol);
-                    tma_load_2d(sm.tiles[stage][1] + bx * kTile * 128, &vmap, &sm.full[stage],
-                                bx * C::kBoxCols, row, pol);
+                    for (int bx = 0; bx < C::kBoxes; ++bx) {
+                        tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128, &kmap, &sm.full[stage],
+                                    bx * C::kBoxCols, row, pol);
+                        tma_load_2d(sm.tiles[stage][1] + bx * kTile * 128, &vmap, &sm.full[stage],
+                                    bx * C::kBoxCols, row, pol);
+                    }
+                } else {
+                    // P-row boxes; rows past the first page are the second page's
+                    const int row2 = (phys2 * a.Hk + kvh) * P;
+                    mbar_arrive_expect_tx(&sm.full[stage], (second ? 2 : 1) * 2 * C::kBoxes * P * 128);
+#pragma unroll
+                    for (int bx = 0; bx < C::kBoxes; ++bx) {
+                        tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128, &kmap, &sm.full[stage],
+                                    bx * C::kBoxCols, row, pol);
+                        tma_load_2d(sm.tiles[stage][1] + bx * kTile * 128, &vmap, &sm.full[stage],
+                                    bx * C::kBoxCols, row, pol);
+                        if (second) {
+                            tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128 + P * 128, &kmap,
+                                        &sm.full[stage], bx * C::kBoxCols, row2, pol);
+                            tma_load_2d(sm.tiles[stage][1] + bx * kTile * 128 + P * 128, &vmap,
+                                        &sm.full[stage], bx * C::kBoxCols, row2, pol);
+                        }
+                    }
                 }
             }
             issued = r + 1;
@@ -991,7 +1027,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
             break;
         }
         const TileRec rec = sm.rec[stage];
-        const float ks = FP8 ? sm.kscale[stage] : 1.f, vs = FP8 ? sm.vscale[stage] : 1.f;
+        const float ks[2] = {FP8 ? sm.kscale[stage][0] : 1.f, FP8 ? sm.kscale[stage][1] : 1.f};
+        const float vs[2] = {FP8 ? sm.vscale[stage][0] : 1.f, FP8 ? sm.vscale[stage][1] : 1.f};
         const int b = rec.b, y = rec.y;
         const int kvh = y / head_chunks, chunk = y % head_chunks;
         const int head_lo = kvh * g + chunk * heads_per_cta;
@@ -1125,7 +1162,9 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &kmap, const CU
     const int g = a.Hq / a.Hk;
     const bool wide = a.pack_gqa && g > 8;
     if (a.kv_dtype == GQA_KV_FP8_E4M3) {
-        if (decode_tile_tokens(a.kv_dtype, a.P) == 32)
+        // 32-token tiles: the balanced schedule on any page size (two boxes on 16-token
+        // pages), the split schedule where a page holds a whole tile
+        if (a.stream_k || decode_tile_tokens(a.kv_dtype, a.P) == 32)
             return wide ? launch_t<128, 2, true, 32>(a, kmap, vmap, stream)
                         : launch_t<128, 1, true, 32>(a, kmap, vmap, stream);
         return wide ? launch_t<128, 2, true, 16>(a, kmap, vmap, stream)
