@@ -16,13 +16,14 @@
 // tcgen05 with P read from tensor memory.
 //
 // Warp roles (384 threads, three warpgroups):
-//   warp 0      TMA producer: both Q tiles (3-D map over [total_q][Hq][D]), then K and V
+//   warp 0      TMA producer: both Q tiles (3-D map over [total_q][Hq][D]), then the K
 //               tiles, 16 keys per copy, gathered page by page through the page table.
 //   warp 1      allocates all 512 tensor-memory columns (S0, S1, O0, O1) and issues the
 //               MMAs from one thread in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so the
 //               tensor core works on one query tile while the other one's softmax runs.
-//   warps 2-3   convert each V tile in place from bf16 to f16 (zeroing keys past the
-//               sequence first), unless a value is beyond the f16 range.
+//   warps 2-3   load the V tiles (warp 2, the same way) and convert each in place from
+//               bf16 to f16 (zeroing keys past the sequence first), unless a value is
+//               beyond the f16 range.
 //   warps 4-7   softmax of query tile 0, warps 8-11 of query tile 1; a thread owns one
 //               row (one tensor-memory lane) and holds its 128 scores in registers.
 // The softmax warpgroups take most of the register file (setmaxnreg).
@@ -179,50 +180,57 @@ __device__ __forceinline__ void softmax_role(PSmem &sm, const PrefillArgs &a, co
                 tmem_st32(tO + 32 * cc, o);
             }
         }
-        // the form P takes depends on whether this V tile became f16
+        // P = 2^(s*c - ref) as f16 value pairs, computed while V tile j may still be
+        // converting (almost every tile becomes f16); the keys of chunk cc go to columns
+        // [32cc, 32cc+16) of S.  Keys go in pairs through the paired fp32 instructions.
+        const unsigned long long c2 = f2_pack(c, c), nref2 = f2_pack(-mref0, -mref0);
+        unsigned long long sum2 = 0ull;  // (0.f, 0.f)
+        uint32_t pk[4][16];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cc][2 * e]),
+                                         __uint_as_float(sr[cc][2 * e + 1])),
+                                 c2, nref2),
+                          x0, x1);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                sum2 = f2_add(sum2, f2_pack(p0, p1));
+                pk[cc][e] = pack_f16(p0, p1);
+            }
+        }
         if (!wait_all(&sm.v_ready[stage], (j / kVStages) & 1)) {
             ok = false;
             break;
         }
         const bool vbf = sm.v_bf16[stage] != 0;
-        // P = 2^(s*c - ref), written over S chunk by chunk: the 32 keys of chunk cc
-        // (columns [32cc, 32cc+32) of S) become 16 columns of value pairs, plus 16 of
-        // residual pairs when the tile stayed bf16.  Keys go in pairs through the
-        // paired fp32 instructions.
-        const unsigned long long c2 = f2_pack(c, c), nref2 = f2_pack(-mref0, -mref0);
-        unsigned long long sum2 = 0ull;  // (0.f, 0.f)
         if (!vbf) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cc][2 * e]),
-                                             __uint_as_float(sr[cc][2 * e + 1])),
-                                     c2, nref2),
-                              x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    sum2 = f2_add(sum2, f2_pack(p0, p1));
-                    pk[e] = pack_f16(p0, p1);
-                }
-                tmem_st16(tS + 32 * cc, pk);
-            }
+            for (int cc = 0; cc < 4; ++cc) tmem_st16(tS + 32 * cc, pk[cc]);
         } else {
+            // the tile stayed bf16: P again from S (not yet overwritten), as bf16 value
+            // pairs in [32cc, 32cc+16) and their bf16 residuals in [32cc+16, 32cc+32)
             const unsigned long long neg1 = f2_pack(-1.f, -1.f);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
+                uint32_t s32[32];
+                tmem_ld32(tS + 32 * cc, s32);
+                tmem_wait_ld();
+                if (nvis < kN) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * cc + e >= nvis) s32[e] = __float_as_uint(-INFINITY);
+                }
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cc][2 * e]),
-                                             __uint_as_float(sr[cc][2 * e + 1])),
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(s32[2 * e]), __uint_as_float(s32[2 * e + 1])),
                                      c2, nref2),
                               x0, x1);
                     const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     const unsigned long long pp = f2_pack(p0, p1);
-                    sum2 = f2_add(sum2, pp);
                     hi[e] = pack_bf16(p0, p1);
                     const unsigned long long hf = f2_pack(__uint_as_float(hi[e] << 16),
                                                           __uint_as_float(hi[e] & 0xffff0000u));
