@@ -1019,6 +1019,16 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     st.reset();
     st.qmul = 1.f;
     int cur_b = -1, cur_y = -1;
+    if (n > 0) {
+        // the first unit's q is loaded while the producer resolves and copies the first tile
+        const FlatPos p0 = flat_locate(s_w, pre, B, U);
+        const int kvh = p0.y / head_chunks, chunk = p0.y % head_chunks;
+        st.load_q(reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                      ((size_t)p0.b * a.Hq + kvh * g + chunk * heads_per_cta) * D,
+                  min(heads_per_cta, g - chunk * heads_per_cta), lane);
+        cur_b = p0.b;
+        cur_y = p0.y;
+    }
     for (long long r = 0; r < n; ++r) {
         const int stage = warp * SW + (int)(r % SW);
         const bool ok = mbar_wait(&sm.full[stage], (uint32_t)((r / SW) & 1));
