@@ -873,6 +873,33 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     const int U = a.Hk * head_chunks;
     const int Lmax = a.pt_stride * P;
 
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        sm.abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kConsumerWarps && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
+    // Everything above may overlap the previous kernel in the stream; the inputs (and the
+    // workspace) are read only after it has completed.
+    grid_dependency_wait();
+    grid_dependents_launch();
+    if (warp == 1) {
+        // the page table into L2 while warp 0 waits for seq_lens: 128-byte lines spread
+        // over the grid, at most 64 per CTA
+        const char *pt0 = reinterpret_cast<const char *>(a.page_table);
+        const long long lines = ((long long)B * a.pt_stride * 4 + 127) / 128;
+        for (long long i = blockIdx.x + (long long)gridDim.x * lane, k = 0; i < lines && k < 2;
+             i += (long long)gridDim.x * 32, ++k)
+            prefetch_l2(pt0 + i * 128);
+    }
+
     // Tiles per sequence and their exclusive prefix (warp 0; lane i owns a run of sequences).
     if (warp == 0) {
         const int per = (B + 31) / 32;
@@ -892,15 +919,6 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
             run += (clamp_len(a.seq_lens[b], Lmax, nullptr) + kTile - 1) / kTile;
         }
         if (lane == 31) pre[B] = incl;
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
-        }
-        sm.abort_flag = 0;
-        fence_barrier_init();
-        fence_proxy_async_smem();
     }
     __syncthreads();
 
@@ -922,10 +940,6 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     if (warp == kConsumerWarps) {
         // ---------------------------------------------- producer: lane w feeds worker w
         if (lane >= kConsumerWarps) return;
-        if (lane == 0) {
-            prefetch_tensormap(&kmap);
-            prefetch_tensormap(&vmap);
-        }
         const uint64_t pol = a.pack_gqa ? policy_evict_first() : policy_evict_last();
         const long long s_w = sk_start(W0cta + lane, T, NW), e_w = sk_start(W0cta + lane + 1, T, NW);
         const long long n = e_w - s_w;
@@ -1153,8 +1167,19 @@ cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtenso
         auto kern = tree ? decode_sk_kernel<D, NT, FP8, TT, true> : decode_sk_kernel<D, NT, FP8, TT, false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<a.grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
-        return cudaGetLastError();
+        // programmatic stream serialization: the kernel's set-up overlaps the tail of the
+        // previous kernel in the stream (the kernel waits for it before reading inputs)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, a, hpc, chunks);
     }
     const size_t smem = sizeof(Smem<D, FP8, kRingSplit, TT>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8, TT>,

@@ -110,6 +110,24 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still running; it
+// must wait (grid_dependency_wait) before it reads or writes global memory that the
+// previous kernel may touch.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel in the stream begin launching (its CTAs still wait for this grid
+// to complete before touching memory).
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Fetch the 128-byte line holding p into L2 (no register result, nothing to wait for).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 // L2 eviction-priority policies for streamed (read-once) and reused data.
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
