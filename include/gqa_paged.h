@@ -125,6 +125,10 @@ int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype)
  *              before first use.  The balanced schedule keeps one merge counter per
  *              (sequence, head) in it, back to zero at the end of every launch; after a
  *              device-side error (see gqa_get_error) zero the workspace again.
+ * The balanced schedule's kernel is launched with programmatic stream serialization: its
+ * CTAs may start (shared-memory set-up only) while the previous kernel on `stream` is
+ * still running, and read or write no global memory until that kernel has completed.
+ * Stream order is therefore kept as for an ordinary launch.
  */
 int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                      const float *k_scale, const float *v_scale, int kv_dtype,
