@@ -225,6 +225,31 @@ def test_repeated_calls_are_deterministic(S):
         assert int(ws[hdr:hdr + 4 * 4 * 32].view(torch.int32).abs().sum()) == 0
 
 
+def test_chained_decodes_read_the_previous_output():
+    """Balanced-schedule launches back to back on one stream, each taking the previous
+    launch's output as its q and sharing one workspace.  A launch may start while the
+    previous kernel is still running (programmatic stream serialization); it must still
+    read the finished output and find the merge counters reset."""
+    import dataclasses
+    case = inputs.llama7b_decode(seed=3)
+    d = to_dev(case)
+    B, Hq, D = case.q.shape
+    ws = binding.new_workspace(binding.gqa_paged_decode_workspace_size(
+        B, Hq, case.Hk, D, 16, d["pt"].shape[1] * 16, 0, 0), DEV)
+    outs, lses = [d["q"]], []
+    for _ in range(3):
+        o, l = binding.gqa_paged_decode(outs[-1], d["k"], d["v"], d["pt"], d["sl"], case.scale,
+                                        workspace=ws)
+        outs.append(o)
+        lses.append(l)
+    torch.cuda.synchronize()
+    assert binding.gqa_get_error(ws) == 0
+    for i in (1, 2):  # launch i + 1 against the oracle on launch i's output
+        ref_o, ref_l = oracle_decode(dataclasses.replace(case, q=outs[i].cpu()))
+        check(outs[i + 1].float().cpu().numpy(), lses[i].cpu().numpy(), ref_o, ref_l,
+              what=f"chained launch {i + 1}")
+
+
 @pytest.mark.parametrize("lens", [[1], [2048], [16] * 37, [0, 0, 5], [3000, 1, 17, 0, 900, 4096]])
 def test_balanced_schedule_shapes(lens):
     """The balanced persistent schedule (num_splits = 0) on batch shapes whose units are
