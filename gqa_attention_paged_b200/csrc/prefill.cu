@@ -596,7 +596,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 }
             }
             const bool big = (mx & 0xffffu) >= kF16Limit || (mx >> 16) >= kF16Limit;
-            // exchange the verdict with the other converter warp: (j + 1) * 2 + flag, and a
+            // exchange the range decision with the other converter warp: (j + 1) * 2 + flag, and a
             // bounded wait for the partner's entry of this tile
             const int mine = ((j + 1) << 1) | (__any_sync(kAll, big) ? 1 : 0);
             volatile int *xo = &sm.conv_ovf[stage][0];
