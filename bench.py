@@ -344,6 +344,8 @@ def main():
     ws = binding.new_workspace(
         binding.gqa_paged_decode_workspace_size(B, Hq, Hk, D, P, pt.shape[1] * P, kvc, S), dev)
     stream = torch.cuda.current_stream(dev)
+    launches = binding.gqa_paged_decode_kernel_launches(B, Hq, Hk, D, P, pt.shape[1] * P, kvc, S,
+                                                        pack)
 
     def step():
         binding.gqa_paged_decode(q, kp, vp, pt, sl, case.scale, num_splits=S, pack_gqa=pack,
@@ -470,7 +472,9 @@ def main():
             "workload": workload_name(a),
             "B_per_gpu": B, "global_batch": B * world, "ctx": a.ctx, "Hq": Hq, "Hk": Hk,
             "head_dim": D, "page_size": P, "num_splits": S, "pack_gqa": pack,
-            "schedule": "balanced persistent (one launch)" if S == 0 else f"{S} splits + merge",
+            "schedule": ("balanced persistent (one launch)" if S == 0 and launches == 1 else
+                         "balanced persistent + merge of cut units (two launches)" if S == 0 else
+                         f"{S} splits + merge"),
             "parallelism": f"dp{world} (independent batches, no collective)",
             "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step per GPU vs 126 MB L2; "
                   "KV loads carry an L2 evict-first hint",
@@ -483,14 +487,15 @@ def main():
                      "unit": "GB/s", "frac": round(kern_gbs / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": ("decode_sk_kernel (the whole call: one launch)" if S == 0 else
+                     "kernel": ("decode_sk_kernel (the whole call: one launch)" if S == 0 and launches == 1 else
+                                "decode_sk_kernel + piece_merge_kernel (the whole call)" if S == 0 else
                                 "decode_kernel (call time minus the separately timed lse_combine)"),
                      "kernel_ms": round(kern_ms, 5), "combine_ms": round(comb_ms, 5)},
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
                 "note": "q, page table and seq_lens H2D from pinned memory, out+lse D2H, "
                         "KV cache device-resident"},
-        "gpu_launches": a.steps * (2 if S > 1 else 1),
+        "gpu_launches": a.steps * launches,
         "clocks": clk,
         "cpu_baseline": cpu,
     }

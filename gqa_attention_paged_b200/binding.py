@@ -37,6 +37,7 @@ SIGNATURES = {
     "gqa_paged_decode_static_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
                                              _I, _I, _I, ctypes.c_float, _I, _I, _P, _P, _P]),
     "gqa_paged_prefill_workspace_size": (_SZ, [_I, _I, _I]),
+    "gqa_paged_decode_kernel_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "gqa_paged_prefill": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                ctypes.c_float, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
@@ -122,6 +123,12 @@ def gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size, max_seq_len,
                                     num_splits) -> int:
     return load().gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size, max_seq_len,
                                                   kv_dtype, num_splits)
+
+
+def gqa_paged_decode_kernel_launches(B, Hq, Hk, head_dim, page_size, max_seq_len, kv_dtype,
+                                     num_splits, pack_gqa=True) -> int:
+    return load().gqa_paged_decode_kernel_launches(B, Hq, Hk, head_dim, page_size, max_seq_len,
+                                                   kv_dtype, num_splits, 1 if pack_gqa else 0)
 
 
 def gqa_paged_prefill_workspace_size(total_q, Hq, head_dim) -> int:

@@ -88,6 +88,15 @@ size_t stream_k_piece_bytes(int Hq, int Hk, int D) {
     return align_up(slots * slot_floats * sizeof(float), 256);
 }
 
+int sm_count();
+
+// CTAs of the balanced decode schedule: kStreamCtasPerSm per SM.
+int decode_grid() {
+    int sms = sm_count();
+    if (sms > kStreamMaxSms) sms = kStreamMaxSms;
+    return sms * kStreamCtasPerSm;
+}
+
 int sm_count() {
     static int cached[256] = {0};
     int dev = 0;
@@ -150,6 +159,18 @@ size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int 
         bytes += align_up((size_t)S * rows * sizeof(float), 256);
     }
     return bytes;
+}
+
+int gqa_paged_decode_kernel_launches(int B, int Hq, int Hk, int head_dim, int page_size,
+                                     int max_seq_len, int kv_dtype, int num_splits,
+                                     int pack_gqa) {
+    (void)head_dim;
+    if (B <= 0 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || page_size <= 0) return 0;
+    if (use_stream_k(num_splits, B))
+        return decode_defers_merge(B, Hq, Hk, pack_gqa ? 1 : 0, decode_grid()) ? 2 : 1;
+    const int S = num_splits > 0 ? num_splits
+                                 : gqa_pick_splits(B, Hk, max_seq_len, page_size, kv_dtype);
+    return S > 1 ? 2 : 1;
 }
 
 size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim) {
@@ -223,11 +244,7 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
     a.stream_k = sk ? 1 : 0;
     a.counters = sk ? reinterpret_cast<int *>(ws + kWorkspaceHeader) : nullptr;
     a.pieces = sk ? reinterpret_cast<float *>(ws + decode_zero_prefix_bytes(B, Hq)) : nullptr;
-    {
-        int sms = sm_count();
-        if (sms > kStreamMaxSms) sms = kStreamMaxSms;
-        a.grid = sms * kStreamCtasPerSm;
-    }
+    a.grid = decode_grid();
     if (launch_decode(a, kmap, vmap, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
     if (S > 1 && launch_lse_combine(a.o_part, a.lse_part, S, (int)rows_q, head_dim, out, lse,
                                     stream) != cudaSuccess)

@@ -18,8 +18,9 @@
 //   - balanced persistent (decode_sk_kernel): a fixed grid; all (sequence, kv head)
 //     tiles are laid end to end and every consumer warp takes an equal contiguous share.
 //     A warp that holds a whole (sequence, kv head) unit writes its output directly; a
-//     unit cut between warps leaves one piece per warp, and the last warp to finish its
-//     piece merges them by log-sum-exp (no second launch).
+//     unit cut between warps leaves one piece per warp.  The last warp to finish its
+//     piece merges them by log-sum-exp in the same launch, or, when units span many
+//     warps (a few long sequences), piece_merge_kernel merges every cut unit after it.
 // Every wait is bounded (2 s): on expiry the kernel records GQA_ERR_TIMEOUT in the
 // workspace error word and returns.
 //
@@ -629,10 +630,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 // merging pieces) never holds up the other warps' streams.
 
 constexpr int kMinTilesPerWorker = 16;
-// A launch whose units average more than this many workers each merges pieces up a
-// tree (the TREE instance); otherwise the last piece of a unit merges all of them.  The
-// two are separate instances so that neither merge's registers burden the other's loop.
-constexpr int kTreeMinWorkersPerUnit = 24;
+// Launches whose units average more than kDeferMinWorkersPerUnit workers each leave their
+// pieces to a second kernel (piece_merge_kernel, the DEFER instance), which merges every
+// cut unit in parallel; otherwise the last piece of a unit to finish merges all of them in
+// the same launch.  The two are separate instances so that the in-launch merge's
+// registers do not burden the other's streaming loop.
 
 __device__ __forceinline__ long long sk_start(long long W, long long T, long long NW) {
     return W >= NW ? T : (W * T) / NW;
@@ -728,130 +730,31 @@ __device__ __forceinline__ void merge_pieces(const float *pieces, long long wfir
     }
 }
 
-// Merge tree for a unit cut into pieces (TREE instance; see the consumer loop):
-// this warp owns leaf `leaf` with its finished state in st; it writes its piece, then
-// climbs while it is the second child to arrive, and the warp reaching the root writes
-// the unit's output.
-template <int D, int NT, bool FP8, int TT, int HW>
-__device__ __forceinline__ void merge_tree(WarpAttn<D, NT, FP8, TT> &st, const DecodeArgs &a,
-                                           long long wfirst, int np, int leaf, int slot_floats,
-                                           int heads_per_cta, int nh, size_t row0, int lane) {
-    using WA = WarpAttn<D, NT, FP8, TT>;
-    constexpr int KT = D / 16;
-    const int gq = lane >> 2, cq = lane & 3;
-    auto slot_of = [&](int leaf) -> float * {
-        return a.pieces + (size_t)((wfirst + leaf) * 2 + (leaf == 0 ? 1 : 0)) * slot_floats;
-    };
-    // own result, normalised, LSE in log2 units
-    float lse2[NT][2];
+// Tiles per sequence and their exclusive prefix into pre[0..B] (one warp; lane i owns a
+// run of sequences).  Lengths are clamped to the page table; err (if not null) records a
+// clamped length.
+template <int TT>
+__device__ __forceinline__ void tile_prefix(const DecodeArgs &a, int *pre, int Lmax, int *err, int lane) {
+    const int B = a.B;
+    const int per = (B + 31) / 32;
+    const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += (clamp_len(a.seq_lens[b], Lmax, err) + TT - 1) / TT;
+    int incl = sum;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-            const float l = st.l[nt][jj];
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            lse2[nt][jj] = l > 0.f ? st.m[nt][jj] + __log2f(l) : -INFINITY;
-#pragma unroll
-            for (int dt = 0; dt < KT; ++dt) {
-                st.o[nt][dt][jj] *= inv;
-                st.o[nt][dt][jj + 2] *= inv;
-            }
-        }
-    auto publish = [&](float *slot) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int h = nt * 8 + 2 * cq + jj;
-                if (h >= nh) continue;
-#pragma unroll
-                for (int dt = 0; dt < KT; ++dt) {
-                    __stcg(slot + h * D + WA::dim0(dt, gq), st.o[nt][dt][jj]);
-                    __stcg(slot + h * D + WA::dim1(dt, gq), st.o[nt][dt][jj + 2]);
-                }
-                if (gq == 0) __stcg(slot + heads_per_cta * D + h, lse2[nt][jj]);
-            }
-        __threadfence();
-        __syncwarp();
-    };
-    // fold the piece at `so` into the registers: left = registers if reg_left
-    auto fold = [&](const float *so, bool reg_left) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int h = nt * 8 + 2 * cq + jj;
-                if (h >= nh) continue;
-                const float ls = __ldcg(so + heads_per_cta * D + h);
-                const float lL = reg_left ? lse2[nt][jj] : ls, lR = reg_left ? ls : lse2[nt][jj];
-                const float M = fmaxf(lL, lR);
-                const float wL = lL == -INFINITY ? 0.f : fast_exp2(lL - M);
-                const float wR = lR == -INFINITY ? 0.f : fast_exp2(lR - M);
-                const float sum = wL + wR;
-                const float inv = sum > 0.f ? 1.f / sum : 0.f;
-                const float cL = wL * inv, cR = wR * inv;
-#pragma unroll
-                for (int dt = 0; dt < KT; ++dt) {
-                    const float s0 = __ldcg(so + h * D + WA::dim0(dt, gq));
-                    const float s1 = __ldcg(so + h * D + WA::dim1(dt, gq));
-                    const float o0 = st.o[nt][dt][jj], o1 = st.o[nt][dt][jj + 2];
-                    const float L0 = reg_left ? o0 : s0, R0 = reg_left ? s0 : o0;
-                    const float L1 = reg_left ? o1 : s1, R1 = reg_left ? s1 : o1;
-                    st.o[nt][dt][jj] = cR == 0.f ? cL * L0 : fmaf(cR, R0, cL * L0);
-                    st.o[nt][dt][jj + 2] = cR == 0.f ? cL * L1 : fmaf(cR, R1, cL * L1);
-                }
-                lse2[nt][jj] = sum > 0.f ? M + __log2f(sum) : -INFINITY;
-            }
-    };
-    int levels = 0;
-    while ((1 << levels) < np) ++levels;
-    int node = leaf, lv = 0;
-    bool mine = true;  // this warp writes the unit's output
-    publish(slot_of(node));
-    while (lv < levels) {
-        const int sib = node ^ 1;
-        if ((sib << lv) >= np) {  // no sibling: the node's result is its parent's
-            node >>= 1;
-            ++lv;
-            continue;
-        }
-        const int p0 = (node >> 1) << (lv + 1);  // parent's leftmost leaf
-        int *ctr = a.counters + ((size_t)((wfirst + p0) * 2 + (p0 == 0 ? 1 : 0)) * kTreeLevels + lv + 1);
-        int second = 0;
-        if (lane == 0) {
-            second = atomicAdd(ctr, 1) == 1;
-            if (second) *ctr = 0;  // ready for the next launch
-        }
-        if (!__shfl_sync(kFull, second, 0)) {
-            mine = false;
-            break;
-        }
-        __threadfence();
-        fold(slot_of(sib << lv), node < sib);
-        node >>= 1;
-        ++lv;
-        if (lv < levels) publish(slot_of(node << lv));
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
     }
-    if (mine) {
-        // the root: the unit's output
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int h = nt * 8 + 2 * cq + jj;
-                if (h >= nh) continue;
-                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) + (row0 + h) * D;
-#pragma unroll
-                for (int dt = 0; dt < KT; ++dt) {
-                    dst[WA::dim0(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj]);
-                    dst[WA::dim1(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj + 2]);
-                }
-                if (gq == 0 && a.lse) a.lse[row0 + h] = lse2[nt][jj] * kLn2;
-            }
+    int run = incl - sum;
+    for (int b = b0; b < b1; ++b) {
+        pre[b] = run;
+        run += (clamp_len(a.seq_lens[b], Lmax, nullptr) + TT - 1) / TT;
     }
+    if (lane == 31) pre[B] = incl;
 }
 
-template <int D, int NT, bool FP8, int TT, bool TREE>
+template <int D, int NT, bool FP8, int TT, bool DEFER>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     decode_sk_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const DecodeArgs a,
@@ -900,26 +803,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
             prefetch_l2(pt0 + i * 128);
     }
 
-    // Tiles per sequence and their exclusive prefix (warp 0; lane i owns a run of sequences).
-    if (warp == 0) {
-        const int per = (B + 31) / 32;
-        const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
-        int sum = 0;
-        for (int b = b0; b < b1; ++b)
-            sum += (clamp_len(a.seq_lens[b], Lmax, blockIdx.x == 0 ? a.err : nullptr) + kTile - 1) / kTile;
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += t;
-        }
-        int run = incl - sum;
-        for (int b = b0; b < b1; ++b) {
-            pre[b] = run;
-            run += (clamp_len(a.seq_lens[b], Lmax, nullptr) + kTile - 1) / kTile;
-        }
-        if (lane == 31) pre[B] = incl;
-    }
+    // Tiles per sequence and their exclusive prefix (warp 0).
+    if (warp == 0) tile_prefix<kTile>(a, pre, Lmax, blockIdx.x == 0 ? a.err : nullptr, lane);
     __syncthreads();
 
     const long long T = (long long)U * pre[B];
@@ -1097,38 +982,32 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
         } else {
             // A piece of a unit shared with neighbouring workers: side 0 = the unit began
             // before this worker's range, side 1 = it begins here and continues after.
-            // Each piece (leaf k = worker wfirst + k) is written normalised with its LSE
-            // (natural log for the flat merge, log2 units in the tree, where a value must not
-            // depend on whether it came through a slot).  Launches whose units span few
-            // workers: the last piece to
-            // finish merges all of them in one pass.  Launches whose units span many
-            // (TREE): the pieces are merged up a binary tree: at level lv, node
-            // n covers leaves [n 2^lv, (n+1) 2^lv); of the two children of a node, the one
-            // whose result is ready second merges the other's (loaded from the slot of its
-            // leftmost leaf) with its own (in registers), left operand first, so the result
-            // does not depend on the order in which workers finish.
+            // The piece is written normalised, with its natural-log LSE.  Launches whose
+            // units span few workers: the last piece to finish merges all of them in one
+            // pass.  Launches whose units span many (DEFER): piece_merge_kernel merges
+            // them after this launch.
             const long long wfirst = sk_worker_of(us, T, NW), wlast = sk_worker_of(ue - 1, T, NW);
             const int np = (int)(wlast - wfirst + 1);
-            if (!TREE) {
-                const int side = us < s_w ? 0 : 1;
-                float *slot = a.pieces + (size_t)(Wme * 2 + side) * slot_floats;
+            const int side = us < s_w ? 0 : 1;
+            float *slot = a.pieces + (size_t)(Wme * 2 + side) * slot_floats;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int h = nt * 8 + 2 * cq + jj;
-                        if (h >= nh) continue;
-                        const float inv = 1.f / st.l[nt][jj];
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int h = nt * 8 + 2 * cq + jj;
+                    if (h >= nh) continue;
+                    const float inv = 1.f / st.l[nt][jj];
 #pragma unroll
-                        for (int dt = 0; dt < KT; ++dt) {
-                            slot[h * D + WA::dim0(dt, gq)] = st.o[nt][dt][jj] * inv;
-                            slot[h * D + WA::dim1(dt, gq)] = st.o[nt][dt][jj + 2] * inv;
-                        }
-                        if (gq == 0) slot[heads_per_cta * D + h] = (st.m[nt][jj] + __log2f(st.l[nt][jj])) * kLn2;
+                    for (int dt = 0; dt < KT; ++dt) {
+                        slot[h * D + WA::dim0(dt, gq)] = st.o[nt][dt][jj] * inv;
+                        slot[h * D + WA::dim1(dt, gq)] = st.o[nt][dt][jj + 2] * inv;
                     }
+                    if (gq == 0) slot[heads_per_cta * D + h] = (st.m[nt][jj] + __log2f(st.l[nt][jj])) * kLn2;
+                }
+            if (!DEFER) {
                 __threadfence();
                 __syncwarp();
-                int *ctr = a.counters + kTreeCounters + (size_t)b * U + y;
+                int *ctr = a.counters + (size_t)b * U + y;
                 int last = 0;
                 if (lane == 0) last = atomicAdd(ctr, 1) == np - 1;
                 last = __shfl_sync(kFull, last, 0);
@@ -1139,13 +1018,97 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
                                         a.lse ? a.lse + row0 : nullptr, lane);
                     if (lane == 0) *ctr = 0;  // ready for the next launch
                 }
-            } else {
-                merge_tree<D, NT, FP8, TT, HW>(st, a, wfirst, np, (int)(Wme - wfirst), slot_floats,
-                                               heads_per_cta, nh, row0, lane);
             }
         }
         st.reset();
         cur_b = -1;
+    }
+}
+
+// Merge of the pieces a DEFER launch of decode_sk_kernel left: one CTA per (unit, head)
+// of a cut unit.  It recomputes the launch's partition (the same tile prefix, worker count
+// and owners), skips units that one worker held whole, and merges pieces wfirst..wlast by
+// log-sum-exp (the merge of NumSplits partials, "解锁GQA性能潜力：从批量大小敏感性到高效优化实践",
+// PackGQA / NumSplits section): the pieces' LSEs go to shared memory in one round of
+// loads; every warp finds M = max lse and W = sum exp(lse - M) there; warp w sums
+// exp(lse_k - M) o_k over pieces k = w, w + 8, ..., eight loads in flight; the eight
+// partial sums are added in warp order.  The result does not depend on which worker
+// finished first.
+constexpr int kMergeWarps = 8;
+
+template <int D, int TT>
+__global__ void __launch_bounds__(32 * kMergeWarps)
+    piece_merge_kernel(const DecodeArgs a, const int heads_per_cta, const int head_chunks) {
+    constexpr int DV = D / 32;
+    __shared__ float part[kMergeWarps][D];
+    __shared__ float lse_s[kStreamMaxWorkers];  // a unit has at most one piece per worker
+    extern __shared__ int pre_m[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int U = a.Hk * head_chunks;
+    const int g = a.Hq / a.Hk;
+    const int h = blockIdx.y;
+    // the pieces are written by the previous kernel in the stream
+    grid_dependency_wait();
+    if (warp == 0) tile_prefix<TT>(a, pre_m, a.pt_stride * a.P, nullptr, lane);
+    __syncthreads();
+    const long long T = (long long)U * pre_m[a.B];
+    const long long NW = min((long long)a.grid * kConsumerWarps, max(1LL, T / kMinTilesPerWorker));
+    const int slot_floats = (heads_per_cta * (D + 1) + 3) & ~3;
+    for (long long u = blockIdx.x; u < (long long)a.B * U; u += gridDim.x) {
+        const int b = (int)(u / U), y = (int)(u % U);
+        const int nt_b = pre_m[b + 1] - pre_m[b];
+        const int kvh = y / head_chunks, chunk = y % head_chunks;
+        const int nh = min(heads_per_cta, g - chunk * heads_per_cta);
+        if (nt_b == 0 || h >= nh) continue;  // uniform for the CTA
+        const long long us = (long long)U * pre_m[b] + (long long)y * nt_b, ue = us + nt_b;
+        const long long wfirst = sk_worker_of(us, T, NW), wlast = sk_worker_of(ue - 1, T, NW);
+        if (wfirst == wlast) continue;  // written whole by its worker
+        const int np = (int)(wlast - wfirst + 1);
+        auto slot = [&](int k) -> const float * {
+            const long long w = wfirst + k;
+            return a.pieces + (size_t)(w * 2 + (k == 0 ? 1 : 0)) * slot_floats;
+        };
+        // every piece's LSE into shared memory, then M and W (each warp, from there)
+        for (int k = threadIdx.x; k < np; k += blockDim.x) lse_s[k] = __ldcg(slot(k) + heads_per_cta * D + h);
+        __syncthreads();
+        float M = -INFINITY;
+        for (int k = lane; k < np; k += 32) M = fmaxf(M, lse_s[k]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+        float W = 0.f;
+        for (int k = lane; k < np; k += 32) W += __expf(lse_s[k] - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(kFull, W, o);
+        // this warp's pieces
+        float acc[DV];
+#pragma unroll
+        for (int v = 0; v < DV; ++v) acc[v] = 0.f;
+#pragma unroll 8
+        for (int k = warp; k < np; k += kMergeWarps) {
+            const float *ps = slot(k);
+            const float wk = __expf(lse_s[k] - M);
+            if constexpr (DV == 4) {
+                const float4 t = __ldcg(reinterpret_cast<const float4 *>(ps + h * D + DV * lane));
+                acc[0] += wk * t.x; acc[1] += wk * t.y; acc[2] += wk * t.z; acc[3] += wk * t.w;
+            } else {
+                const float2 t = __ldcg(reinterpret_cast<const float2 *>(ps + h * D + DV * lane));
+                acc[0] += wk * t.x; acc[1] += wk * t.y;
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < DV; ++v) part[warp][DV * lane + v] = acc[v];
+        __syncthreads();
+        const int head_lo = kvh * g + chunk * heads_per_cta;
+        const float inv = 1.f / W;
+        for (int d = threadIdx.x; d < D; d += blockDim.x) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kMergeWarps; ++w) sum += part[w][d];
+            reinterpret_cast<__nv_bfloat16 *>(a.out)[((size_t)b * a.Hq + head_lo + h) * D + d] =
+                __float2bfloat16(sum * inv);
+        }
+        if (threadIdx.x == 0 && a.lse) a.lse[(size_t)b * a.Hq + head_lo + h] = M + logf(W);
+        __syncthreads();  // part[] and lse_s[] are reused by the next unit
     }
 }
 
@@ -1162,9 +1125,8 @@ cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtenso
     if (a.stream_k) {
         const size_t smem =
             sizeof(Smem<D, FP8, kRingBalanced, TT>) + 1024 + sizeof(int) * (size_t)(a.B + 1);
-        const long long units = (long long)a.B * a.Hk * chunks;
-        const bool tree = (long long)a.grid * kConsumerWarps > kTreeMinWorkersPerUnit * units;
-        auto kern = tree ? decode_sk_kernel<D, NT, FP8, TT, true> : decode_sk_kernel<D, NT, FP8, TT, false>;
+        const bool defer = decode_defers_merge(a.B, a.Hq, a.Hk, a.pack_gqa, a.grid);
+        auto kern = defer ? decode_sk_kernel<D, NT, FP8, TT, true> : decode_sk_kernel<D, NT, FP8, TT, false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         // programmatic stream serialization: the kernel's set-up overlaps the tail of the
@@ -1179,7 +1141,15 @@ cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtenso
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, a, hpc, chunks);
+        e = cudaLaunchKernelEx(&cfg, kern, kmap, vmap, a, hpc, chunks);
+        if (e != cudaSuccess || !defer) return e;
+        // the merge of the cut units: an ordinary launch (measured faster than letting its
+        // CTAs wait beside the decode kernel's)
+        const long long nunits = (long long)a.B * a.Hk * chunks;
+        piece_merge_kernel<D, TT><<<dim3((unsigned)(nunits < 4096 ? nunits : 4096), (unsigned)hpc),
+                                    32 * kMergeWarps, sizeof(int) * (size_t)(a.B + 1), stream>>>(
+            a, hpc, chunks);
+        return cudaGetLastError();
     }
     const size_t smem = sizeof(Smem<D, FP8, kRingSplit, TT>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8, TT>,

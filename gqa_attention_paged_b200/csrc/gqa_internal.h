@@ -28,7 +28,7 @@ struct DecodeArgs {
     int *err;
     // balanced persistent schedule (num_splits == 0, B <= kStreamMaxBatch)
     int stream_k;
-    int *counters;  // [2 * workers][kTreeLevels] tree, then [B * units] flat merge counters; zero between launches
+    int *counters;  // [B * units] merge counters of the last-piece merge; zero between launches
     float *pieces;  // [workers * 2][heads per CTA][D + 1]
     int grid;       // persistent CTAs
 };
@@ -41,20 +41,33 @@ constexpr int kStreamCtasPerSm = 2;
 constexpr int kStreamMaxSms = 160;
 constexpr int kStreamWorkersPerCta = 4;
 
-// Levels of the balanced schedule's merge tree (pieces per unit <= workers < 2^11).
-constexpr int kTreeLevels = 12;
 constexpr int kStreamMaxWorkers = kStreamMaxSms * kStreamCtasPerSm * kStreamWorkersPerCta;
 
-// Bytes at the start of a decode workspace that must be zero before a launch: the error
-// word header, then the balanced schedule's merge counters: one per (piece slot, tree
-// level) for 2 slots per worker of the largest grid, then one per (sequence, head) for
-// units merged by their last piece.
-constexpr size_t kTreeCounters = (size_t)2 * kStreamMaxWorkers * kTreeLevels;
-inline size_t decode_zero_prefix_bytes(int B, int Hq) {
-    return kWorkspaceHeader + ((kTreeCounters + (size_t)B * Hq) * sizeof(int) + 255) / 256 * 256;
+// Packed query heads per decode CTA: the whole group with PackGQA (up to 16, the wide
+// instance for groups above 8), else one head.
+inline int decode_heads_per_cta(int Hq, int Hk, int pack_gqa) {
+    const int g = Hq / Hk;
+    const int cap = g > 8 ? 16 : 8;
+    return pack_gqa ? (g < cap ? g : cap) : 1;
+}
+// A balanced-schedule launch whose units average more than this many workers each leaves
+// its pieces to a second kernel, which merges every cut unit in parallel; otherwise the
+// last piece of each unit merges the unit in the same launch.
+constexpr int kDeferMinWorkersPerUnit = 24;
+inline bool decode_defers_merge(int B, int Hq, int Hk, int pack_gqa, int grid) {
+    const int g = Hq / Hk, hpc = decode_heads_per_cta(Hq, Hk, pack_gqa);
+    const long long units = (long long)B * Hk * ((g + hpc - 1) / hpc);
+    return (long long)grid * kStreamWorkersPerCta > (long long)kDeferMinWorkersPerUnit * units;
 }
 
-// Launch the decode kernel (and nothing else) on `stream`.  The tensor maps describe the
+// Bytes at the start of a decode workspace that must be zero before a launch: the error
+// word header, then the balanced schedule's merge counters, one per (sequence, head).
+inline size_t decode_zero_prefix_bytes(int B, int Hq) {
+    return kWorkspaceHeader + ((size_t)B * Hq * sizeof(int) + 255) / 256 * 256;
+}
+
+// Launch the decode kernel on `stream` (for launches whose units are cut into many pieces,
+// followed by the kernel that merges the pieces).  The tensor maps describe the
 // K and V pools as 2-D arrays [num_pages*Hk*P rows][D].
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);

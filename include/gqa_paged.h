@@ -80,11 +80,22 @@ typedef enum {
  * header holding the device error word, then
  *   num_splits = 0, B <= 2048 (balanced schedule): int32 merge counters [B*Hq] (rounded
  *     up to 256 bytes) and the merge pieces, 2 per worker of the largest grid
- *     (160 SMs x 3 CTAs x 4 workers), each min(Hq/Hk, 16) x (head_dim + 1) fp32;
+ *     (160 SMs x 2 CTAs x 4 workers), each min(Hq/Hk, 16) x (head_dim + 1) fp32;
  *   split schedule with S > 1: o_part fp32 [S][B*Hq][head_dim] and lse_part fp32 [S][B*Hq].
  */
 size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int page_size,
                                        int max_seq_len, int kv_dtype, int num_splits);
+
+/*
+ * Kernels one gqa_paged_decode() call with these arguments launches on the current
+ * device: 1, or 2 when a second kernel merges partial results (split schedule with
+ * S > 1: lse_combine; balanced schedule when its units average more than 24 workers
+ * each, e.g. a few long sequences: the kernel that merges the pieces of cut units).
+ * Returns 0 for sizes gqa_paged_decode() rejects.  Host only; launches nothing.
+ */
+int gqa_paged_decode_kernel_launches(int B, int Hq, int Hk, int head_dim, int page_size,
+                                     int max_seq_len, int kv_dtype, int num_splits,
+                                     int pack_gqa);
 
 /*
  * Split count gqa_paged_decode() uses with num_splits = 0 when B is above the balanced

@@ -33,6 +33,17 @@ def test_header_declares_the_boundary():
         assert n in names, n
 
 
+def test_decode_kernel_launch_count():
+    """Host-only policy: one launch, or two when a second kernel merges partial results."""
+    f = binding.gqa_paged_decode_kernel_launches
+    assert f(64, 32, 8, 128, 16, 2048, 0, 0) == 1          # balanced, in-launch merge
+    assert f(4, 64, 8, 128, 64, 32768, 0, 0) == 2          # few long sequences: merge kernel
+    assert f(64, 32, 8, 128, 16, 2048, 0, 1) == 1          # one split
+    assert f(64, 32, 8, 128, 16, 2048, 0, 4) == 2          # splits + lse_combine
+    assert f(0, 32, 8, 128, 16, 2048, 0, 0) == 0           # rejected sizes
+    assert f(4, 30, 8, 128, 16, 2048, 0, 0) == 0
+
+
 def test_library_exports_every_declared_symbol():
     lib = binding.load()
     for name in declared_functions():

@@ -4,8 +4,9 @@ share.  The formulas are the ones decode_sk_kernel evaluates (restated here): wo
 owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // 16)); the owner
 of tile t is ((t+1)*NW + T-1)//T - 1;
 a unit cut between workers leaves one piece per worker, side 1 for the worker where the
-unit begins and side 0 for the others; the pieces are merged up a binary tree whose
-internal nodes are claimed by the second of their two children to arrive."""
+unit begins and side 0 for the others.  The last piece of a unit merges them in the same
+launch, or, for launches whose units span many workers, a separate merge kernel reads the
+same slots."""
 import itertools
 import random
 
@@ -112,66 +113,59 @@ def test_slot_indices_stay_in_the_workspace():
         assert 2 * (workers - 1) + 1 < 2 * workers
 
 
-def tree_merge(np_, order, levels_cap=12):
-    """Replay the merge-tree protocol for np_ pieces whose leaf owners finish in `order`.
-    Each owner climbs: no sibling -> move up; else arrive at the parent's counter; the
-    first arrival stops, the second merges (left operand first) and climbs on.  Returns
-    the root's operand tree and the counter ids used."""
-    levels = 0
-    while (1 << levels) < np_:
-        levels += 1
-    assert levels < levels_cap
-    counters, results, roots, used = {}, {k: k for k in range(np_)}, [], set()
-    pending = {}
-    for k in order:
-        node, lv, val = k, 0, k
-        while lv < levels:
-            sib = node ^ 1
-            if (sib << lv) >= np_:
-                node >>= 1
-                lv += 1
-                continue
-            p0 = (node >> 1) << (lv + 1)
-            cid = (p0, lv + 1)
-            used.add(cid)
-            counters[cid] = counters.get(cid, 0) + 1
-            if counters[cid] == 1:
-                pending[(lv, node)] = val
-                break
-            other = pending.pop((lv, sib))
-            val = (val, other) if node < sib else (other, val)
-            node >>= 1
-            lv += 1
-        else:
-            roots.append(val)
-    return roots, counters, used
+def defers(B, Hq, Hk, pack, grid):
+    """The host policy (decode_defers_merge): units averaging more than 24 workers each
+    leave their pieces to the separate merge kernel."""
+    g = Hq // Hk
+    hpc = (min(g, 16 if g > 8 else 8)) if pack else 1
+    units = B * Hk * ((g + hpc - 1) // hpc)
+    return grid * 4 > 24 * units
 
 
-def _tree_of(np_):
-    levels = 0
-    while (1 << levels) < np_:
-        levels += 1
-    def build(lv, node):
-        lo = node << lv
-        if lo >= np_:
-            return None
-        if lv == 0:
-            return lo
-        l, r = build(lv - 1, 2 * node), build(lv - 1, 2 * node + 1)
-        return l if r is None else (l, r)
-    return build(levels, 0)
+def merge_kernel_reads(tiles_per_seq, U, workers):
+    """The piece slots the merge kernel reads per unit: pieces of workers wfirst..wlast,
+    slot W*2 + (1 if W == wfirst else 0), for units held by more than one worker."""
+    pre = [0]
+    for n in tiles_per_seq:
+        pre.append(pre[-1] + n)
+    T = U * pre[-1]
+    NW = n_workers(workers, T)
+    reads = {}
+    for b, n in enumerate(tiles_per_seq):
+        if n == 0:
+            continue
+        for y in range(U):
+            us = U * pre[b] + y * n
+            w0, w1 = owner(us, T, NW), owner(us + n - 1, T, NW)
+            if w0 != w1:
+                reads[(b, y)] = sorted([(w0, 1)] + [(W, 0) for W in range(w0 + 1, w1 + 1)])
+    return reads
 
 
-@pytest.mark.parametrize("np_", [2, 3, 4, 5, 7, 8, 9, 16, 37, 100, 1280])
-def test_merge_tree_has_one_root_and_a_fixed_shape(np_):
-    rng = random.Random(np_)
-    want = _tree_of(np_)
-    for trial in range(20):
-        order = list(range(np_))
-        rng.shuffle(order)
-        roots, counters, used = tree_merge(np_, order)
-        assert len(roots) == 1, "exactly one worker writes the unit"
-        assert roots[0] == want, "the result must not depend on the arrival order"
-        assert all(c == 2 for c in counters.values()), "every counter is claimed by two children"
-        # counter ids stay inside [2 * workers][12]: leaf slot < 2 * 1280, level < 12
-        assert all(p0 < 1280 and 1 <= lv < 12 for p0, lv in used)
+@pytest.mark.parametrize("workers", [4, 64, 1184])
+def test_merge_kernel_reads_exactly_the_written_pieces(workers):
+    """For every cut unit, the separate merge kernel reads exactly the slots the workers
+    wrote, and no slot is written for two units."""
+    rng = random.Random(workers)
+    for trial in range(12):
+        B = rng.randint(1, 6)
+        tiles = [rng.choice([0, 1, 3, 64, 512]) for _ in range(B)]
+        U = rng.choice([1, 8])
+        _, _, _, pieces = schedule(tiles, U, workers)
+        reads = merge_kernel_reads(tiles, U, workers)
+        assert set(reads) == set(pieces), (tiles, U)
+        seen = set()
+        for key, slots in reads.items():
+            assert slots == sorted(pieces[key]), (tiles, U, key)
+            for s_ in slots:
+                assert s_ not in seen
+                seen.add(s_)
+
+
+def test_defer_policy_on_the_named_shapes():
+    grid = 148 * 2
+    assert defers(4, 64, 8, True, grid)        # 70B long context: 32 units, 37 workers each
+    assert defers(1, 32, 8, True, grid)        # one sequence
+    assert not defers(64, 32, 8, True, grid)   # B=64 sweep: 2 workers per unit
+    assert not defers(16, 32, 8, True, grid)   # 7B-shaped batch
+    assert not defers(8, 32, 8, False, grid)   # PackGQA off: one unit per head
