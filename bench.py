@@ -200,6 +200,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--append", action="store_true",
+                    help="decode workloads: time gqa_paged_append_decode (each step first "
+                         "writes the new token's K/V into its page)")
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "long70b"],
                     help="decode: the headline (paged GQA decode); prefill: causal chunked "
                          "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]; "
@@ -210,8 +213,8 @@ def parse():
 def workload_name(a):
     if a.workload == "long70b":
         return f"paged GQA decode, 70B-shaped long context: B=4 ctx={{8K,16K,24K,32K}} Hq=64 Hk=8 D=128 page_size=64 kv={a.kv}"
-    return (f"paged GQA decode, B={a.B} ctx={a.ctx} Hq=32 Hk=8 D=128 page_size=16 "
-            f"kv={a.kv}")
+    return (f"paged GQA {'KV append + ' if a.append else ''}decode, B={a.B} ctx={a.ctx} Hq=32 "
+            f"Hk=8 D=128 page_size=16 kv={a.kv}")
 
 
 def prefill_flops(prior_lens, q_lens, Hq, D):
@@ -346,8 +349,19 @@ def main():
     stream = torch.cuda.current_stream(dev)
     launches = binding.gqa_paged_decode_kernel_launches(B, Hq, Hk, D, P, pt.shape[1] * P, kvc, S,
                                                         pack)
+    if a.append:
+        # the new token of every sequence (position seq_len - 1), written before each decode
+        gk = torch.Generator().manual_seed(a.seed + 1)
+        k_new = torch.randn(B, Hk, D, generator=gk).to(torch.bfloat16).to(dev)
+        v_new = torch.randn(B, Hk, D, generator=gk).to(torch.bfloat16).to(dev)
+        launches += 1
 
     def step():
+        if a.append:
+            binding.gqa_paged_append_decode(q, k_new, v_new, kp, vp, pt, sl, case.scale,
+                                            num_splits=S, pack_gqa=pack, k_scale=ks, v_scale=vs,
+                                            out=out, lse=lse, workspace=ws, stream=stream)
+            return
         binding.gqa_paged_decode(q, kp, vp, pt, sl, case.scale, num_splits=S, pack_gqa=pack,
                                  k_scale=ks, v_scale=vs, out=out, lse=lse, workspace=ws,
                                  stream=stream)
@@ -434,6 +448,8 @@ def main():
 
     lens = [int(x) for x in kv.seq_lens]
     step_bytes = decode_step_bytes(lens, Hq, Hk, D, elem, P)
+    if a.append:  # the new tokens' K/V read (bf16) and written into the pages
+        step_bytes += 2 * B * Hk * D * (2 + elem)
     peak, peak_kind = peaks()
     gbs = aggregate_gbs(step_bytes, world, ms)
     kern_gbs = step_bytes / (kern_ms * 1e-3) / 1e9

@@ -42,6 +42,10 @@ SIGNATURES = {
                                ctypes.c_float, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "gqa_paged_gather": (_I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "gqa_paged_append_kv": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I,
+                                 _P, _P]),
+    "gqa_paged_append_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
+                                     _I, _I, _I, ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
     "gqa_get_error": (_I, [_P, _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -222,6 +226,84 @@ def gqa_paged_decode_static_scratch(q: torch.Tensor, k_pages: torch.Tensor,
         float(scale), int(num_splits), int(bool(pack_gqa)), _ptr(out), _ptr(lse),
         _stream(stream))
     _check("gqa_paged_decode_static_scratch", st)
+    return out, lse
+
+
+def _append_args(k_new, v_new, k_pages, v_pages, page_table, seq_lens, k_scale, v_scale):
+    _need(k_pages, "k_pages", _KV_DTYPES)
+    _need(v_pages, "v_pages", k_pages.dtype, k_pages.shape)
+    num_pages, Hk, P, D = k_pages.shape
+    _need(seq_lens, "seq_lens", torch.int32)
+    B = seq_lens.shape[0]
+    _need(k_new, "k_new", torch.bfloat16, (B, Hk, D))
+    _need(v_new, "v_new", torch.bfloat16, (B, Hk, D))
+    _need(page_table, "page_table", torch.int32)
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B][pt_stride]")
+    kv_dtype = _kv_code(k_pages)
+    if kv_dtype == GQA_KV_FP8_E4M3:
+        if k_scale is None or v_scale is None:
+            raise ValueError("fp8 KV needs k_scale and v_scale")
+        _need(k_scale, "k_scale", torch.float32, (num_pages, Hk))
+        _need(v_scale, "v_scale", torch.float32, (num_pages, Hk))
+    return B, Hk, D, P, num_pages, kv_dtype
+
+
+def gqa_paged_append_kv(k_new: torch.Tensor, v_new: torch.Tensor, k_pages: torch.Tensor,
+                        v_pages: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
+                        k_scale: Optional[torch.Tensor] = None,
+                        v_scale: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Write token seq_lens[b] - 1 of every sequence (k_new / v_new bf16 [B][Hk][D]) into
+    the paged cache, in place (e4m3 pools quantise it; see include/gqa_paged.h).  Returns
+    the workspace holding the error word."""
+    B, Hk, D, P, num_pages, kv_dtype = _append_args(k_new, v_new, k_pages, v_pages, page_table,
+                                                     seq_lens, k_scale, v_scale)
+    if workspace is None:
+        workspace = new_workspace(256, k_pages.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = load().gqa_paged_append_kv(
+        _ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale),
+        kv_dtype, _ptr(page_table), page_table.shape[1], _ptr(seq_lens), B, Hk, D, P, num_pages,
+        _ptr(workspace), _stream(stream))
+    _check("gqa_paged_append_kv", st)
+    return workspace
+
+
+def gqa_paged_append_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                            k_pages: torch.Tensor, v_pages: torch.Tensor,
+                            page_table: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                            num_splits: int = 0, pack_gqa: bool = True,
+                            k_scale: Optional[torch.Tensor] = None,
+                            v_scale: Optional[torch.Tensor] = None,
+                            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None, want_lse: bool = True,
+                            stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """gqa_paged_append_kv then gqa_paged_decode on one stream."""
+    _need(q, "q", torch.bfloat16)
+    B, Hk, D, P, num_pages, kv_dtype = _append_args(k_new, v_new, k_pages, v_pages, page_table,
+                                                     seq_lens, k_scale, v_scale)
+    Bq, Hq, Dq = q.shape
+    if Bq != B or Dq != D:
+        raise ValueError("q must be [B][Hq][head_dim] with the pools' head_dim")
+    pt_stride = page_table.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq))
+    need = gqa_paged_decode_workspace_size(B, Hq, Hk, D, P, pt_stride * P, kv_dtype, num_splits)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = load().gqa_paged_append_decode(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale),
+        _ptr(v_scale), kv_dtype, _ptr(page_table), pt_stride, _ptr(seq_lens), B, Hq, Hk, D, P,
+        num_pages, float(scale), int(num_splits), int(bool(pack_gqa)), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("gqa_paged_append_decode", st)
     return out, lse
 
 

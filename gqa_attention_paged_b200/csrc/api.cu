@@ -343,6 +343,72 @@ int gqa_paged_gather(const void *k_pages, const void *v_pages, const int32_t *pa
                : GQA_ERR_LAUNCH;
 }
 
+int gqa_paged_append_kv(const void *k_new, const void *v_new, void *k_pages, void *v_pages,
+                        float *k_scale, float *v_scale, int kv_dtype, const int32_t *page_table,
+                        int pt_stride, const int32_t *seq_lens, int B, int Hk, int head_dim,
+                        int page_size, int num_pages, void *workspace, cudaStream_t stream) {
+    if (!k_new || !v_new || !k_pages || !v_pages || !page_table || !seq_lens || !workspace)
+        return GQA_ERR_NULL;
+    if (kv_dtype != GQA_KV_BF16 && kv_dtype != GQA_KV_FP8_E4M3) return GQA_ERR_DTYPE;
+    if (kv_dtype == GQA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return GQA_ERR_DTYPE;
+    if (B < 0 || B > 65535 || Hk <= 0 || Hk > 65535 || (head_dim != 64 && head_dim != 128) ||
+        !valid_page_size(page_size) || num_pages <= 0 || pt_stride <= 0 ||
+        (int64_t)num_pages * Hk * page_size > INT32_MAX ||
+        (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (!aligned(k_new, 2) || !aligned(v_new, 2) || !aligned(k_pages, 2) ||
+        !aligned(v_pages, 2) || !aligned(page_table, 4) || !aligned(seq_lens, 4) ||
+        !aligned(workspace, 256) || (k_scale && !aligned(k_scale, 4)) ||
+        (v_scale && !aligned(v_scale, 4)))
+        return GQA_ERR_ALIGN;
+    AppendArgs a;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.k_pages = k_pages;
+    a.v_pages = v_pages;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.kv_dtype = kv_dtype;
+    a.page_table = page_table;
+    a.pt_stride = pt_stride;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.Hk = Hk;
+    a.D = head_dim;
+    a.P = page_size;
+    a.num_pages = num_pages;
+    a.err = reinterpret_cast<int *>(workspace);
+    return launch_append(a, stream) == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
+}
+
+int gqa_paged_append_decode(const void *q, const void *k_new, const void *v_new, void *k_pages,
+                            void *v_pages, float *k_scale, float *v_scale, int kv_dtype,
+                            const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                            int B, int Hq, int Hk, int head_dim, int page_size, int num_pages,
+                            float scale, int num_splits, int pack_gqa, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    // the decode's checks first, so that a call it would reject changes nothing
+    if (!q || !out) return GQA_ERR_NULL;
+    if (Hq <= 0 || Hk <= 0 || Hq % Hk != 0) return GQA_ERR_SHAPE;
+    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (kv_dtype == GQA_KV_FP8_E4M3 && head_dim != 128) return GQA_ERR_DTYPE;
+    if (!workspace || !aligned(workspace, 256)) return workspace ? GQA_ERR_WORKSPACE : GQA_ERR_NULL;
+    const bool sk = use_stream_k(num_splits, B);
+    const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
+    if (workspace_bytes < gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                          pt_stride * page_size, kv_dtype,
+                                                          sk ? 0 : S))
+        return GQA_ERR_WORKSPACE;
+    const int r = gqa_paged_append_kv(k_new, v_new, k_pages, v_pages, k_scale, v_scale,
+                                      kv_dtype, page_table, pt_stride, seq_lens, B, Hk,
+                                      head_dim, page_size, num_pages, workspace, stream);
+    if (r != GQA_OK) return r;
+    return gqa_paged_decode(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table,
+                            pt_stride, seq_lens, B, Hq, Hk, head_dim, page_size, num_pages,
+                            scale, num_splits, pack_gqa, out, lse, workspace, workspace_bytes,
+                            stream);
+}
+
 int gqa_get_error(void *workspace, cudaStream_t stream) {
     if (!workspace) return GQA_ERR_NULL;
     int err = 0;

@@ -109,6 +109,20 @@ cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap,
                            const CUtensorMap &vmap, const CUtensorMap &qmap,
                            cudaStream_t stream);
 
+// KV append: the new token of each sequence into its page (append.cu).
+struct AppendArgs {
+    const void *k_new, *v_new;  // bf16 [B][Hk][D]
+    void *k_pages, *v_pages;
+    float *k_scale, *v_scale;   // e4m3 only
+    int kv_dtype;
+    const int32_t *page_table;
+    int pt_stride;
+    const int32_t *seq_lens;
+    int B, Hk, D, P, num_pages;
+    int *err;
+};
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t stream);
+
 // Tokens per decode pipeline stage (the TMA box height of the KV tensor maps): 32 for
 // e4m3 KV on pages of at least 32 tokens, else 16.
 inline int decode_tile_tokens(int kv_dtype, int page_size) {

@@ -238,6 +238,45 @@ int lse_combine(const float *o_part, const float *lse_part, int num_splits, int 
                 int head_dim, void *out, float *lse, cudaStream_t stream);
 
 /*
+ * KV append: writes each sequence's new token into the paged cache, the step before decode
+ * (the fused decoder step of "FasterTransformer source tour" counts this write among its
+ * three global accesses).  seq_lens[b] already counts the new token, so token L_b - 1 of
+ * sequence b goes to page page_table[b][(L_b - 1) / page_size], slot (L_b - 1) % page_size,
+ * for every kv head j:
+ *   bf16 pools:  k_pages[...][j][slot][:] = k_new[b][j][:] (bits copied), same for v.
+ *   e4m3 pools:  a token that opens a page (slot 0) sets k_scale[page][j] = absmax / 448
+ *                (fp32; 1 for an all-zero token), a later token keeps the page's scale;
+ *                each element is stored as e4m3(x / scale), the fp32 quotient rounded to
+ *                nearest even and saturated at +-448.  The same for v.
+ * Sequences with seq_lens[b] = 0 append nothing.
+ *
+ *   k_new, v_new  bf16 [B][Hk][head_dim]
+ *   k_pages, v_pages, page_table, seq_lens, page sizes: as for gqa_paged_decode()
+ *   k_scale, v_scale  fp32 [num_pages][Hk], read and written for GQA_KV_FP8_E4M3
+ *   workspace   >= 256 bytes, 256-byte aligned; its error word records a page-table
+ *               entry or seq_len out of range (that token is not written)
+ * Two sequences whose new tokens fall on the same (page, slot) race.
+ */
+int gqa_paged_append_kv(const void *k_new, const void *v_new, void *k_pages, void *v_pages,
+                        float *k_scale, float *v_scale, int kv_dtype, const int32_t *page_table,
+                        int pt_stride, const int32_t *seq_lens, int B, int Hk, int head_dim,
+                        int page_size, int num_pages, void *workspace, cudaStream_t stream);
+
+/*
+ * gqa_paged_append_kv() then gqa_paged_decode() on the same stream: the new token of every
+ * sequence is written into its page, then attended to with the rest of the history.
+ * Arguments are the two calls'; the decode's checks run first, so a rejected call
+ * changes nothing.  The decode kernel starts its set-up while the append kernel finishes
+ * and reads the cache only after it has completed.
+ */
+int gqa_paged_append_decode(const void *q, const void *k_new, const void *v_new, void *k_pages,
+                            void *v_pages, float *k_scale, float *v_scale, int kv_dtype,
+                            const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                            int B, int Hq, int Hk, int head_dim, int page_size, int num_pages,
+                            float scale, int num_splits, int pack_gqa, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Copy-out of the paged cache into contiguous per-sequence storage, bit for bit:
  *   k_out[cu_kv[b] + t][j][:] = k_pages[page_table[b][t / page_size]][j][t % page_size][:]
  * and the same for v, for t < seq_lens[b].  elem_bytes is 2 (bf16) or 1 (fp8); bytes

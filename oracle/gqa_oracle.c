@@ -350,3 +350,88 @@ int oracle_num_threads(void)
     }
     return n;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * KV append (the step before decode: "FasterTransformer source tour", where the fused
+ * decoder step counts writing the new token into the KV cache among its three global
+ * accesses; page layout as above).  Readings taken where the pages are silent:
+ *   - seq_lens[b] already counts the new token, so it goes to position L_b - 1: page
+ *     page_table[b][(L_b - 1) / P], slot (L_b - 1) % P, for every kv head.  L_b = 0
+ *     appends nothing.
+ *   - bf16 pools take the token's bits as given.
+ *   - e4m3 pools: a token that opens a page (slot 0) sets that (page, kv head)'s scale
+ *     to absmax / 448 in fp32 (1 for an all-zero token); a later token keeps the page's
+ *     scale.  Each element becomes e4m3(x / scale), the quotient in fp32, rounded to
+ *     nearest (ties to even) and saturated at +-448.
+ * ------------------------------------------------------------------------------------- */
+
+/* OCP e4m3 code of x: the nearest of the 127 non-negative finite codes by exhaustive
+ * search (ties to the even code, i.e. mantissa LSB 0), with x's sign; magnitudes past 448
+ * and infinities give +-448; NaN gives the NaN code 0x7f. */
+uint8_t oracle_f32_to_e4m3(float x)
+{
+    if (isnan(x))
+        return 0x7f;
+    int sign = signbit(x) ? 1 : 0;
+    if (isinf(x))
+        return (uint8_t)((sign << 7) | 0x7e);
+    double ax = fabs((double)x);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= 0x7e; ++c) {
+        double d = fabs(oracle_e4m3_to_f64((uint8_t)c) - ax);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            bd = d;
+            best = c;
+        }
+    }
+    return (uint8_t)((sign << 7) | best);
+}
+
+static float bf16_bits_to_f32(uint16_t bits)
+{
+    return (float)oracle_bf16_to_f64(bits); /* exact: bf16 is a truncated binary32 */
+}
+
+void oracle_append_kv(void *k_pages, void *v_pages, float *k_scale, float *v_scale,
+                      int kv_dtype, const int32_t *page_table, int pt_stride,
+                      const int32_t *seq_lens, int B, int Hk, int D, int P,
+                      const uint16_t *k_new, const uint16_t *v_new)
+{
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        if (L <= 0)
+            continue;
+        int t = L - 1;
+        int64_t phys = page_table[(int64_t)b * pt_stride + t / P];
+        int slot = t % P;
+        for (int kvh = 0; kvh < Hk; ++kvh) {
+            for (int which = 0; which < 2; ++which) {
+                const uint16_t *src = (which == 0 ? k_new : v_new) + ((int64_t)b * Hk + kvh) * D;
+                void *pages = which == 0 ? k_pages : v_pages;
+                int64_t base = (((phys * Hk) + kvh) * (int64_t)P + slot) * D;
+                if (kv_dtype == 0) {
+                    for (int d = 0; d < D; ++d)
+                        ((uint16_t *)pages)[base + d] = src[d];
+                    continue;
+                }
+                float *scale = which == 0 ? k_scale : v_scale;
+                int64_t si = phys * Hk + kvh;
+                if (slot == 0) {
+                    float amax = 0.0f;
+                    for (int d = 0; d < D; ++d) {
+                        float a = fabsf(bf16_bits_to_f32(src[d]));
+                        if (a > amax)
+                            amax = a;
+                    }
+                    scale[si] = amax > 0.0f ? amax / 448.0f : 1.0f;
+                }
+                float s = scale[si];
+                for (int d = 0; d < D; ++d) {
+                    float qv = bf16_bits_to_f32(src[d]) / s;
+                    ((uint8_t *)pages)[base + d] = oracle_f32_to_e4m3(qv);
+                }
+            }
+        }
+    }
+}

@@ -47,6 +47,12 @@ def lib():
                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
                                      _P, _P]
         L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+        L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.oracle_append_kv.restype = None
+        L.oracle_append_kv.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _P, _P]
         _lib = L
     return _lib
 
@@ -193,3 +199,31 @@ class use_library:
         global _lib
         _lib = self.saved
         return False
+
+
+def f32_to_e4m3(x):
+    """e4m3 codes of fp32 values (round to nearest even, saturating at +-448)."""
+    f = lib().oracle_f32_to_e4m3
+    a = np.asarray(x, np.float32)
+    return np.array([f(float(v)) for v in a.ravel()], np.uint8).reshape(a.shape)
+
+
+def append_kv(k_pages, v_pages, page_table, seq_lens, k_new, v_new, k_scale=None, v_scale=None):
+    """Copies of the pools (and scales) with token seq_lens[b] - 1 of every sequence
+    written from k_new / v_new (bf16 bits [B][Hk][D]); e4m3 pools quantise it (see
+    oracle_append_kv).  Returns (k_pages, v_pages, k_scale, v_scale)."""
+    kp = np.array(k_pages, copy=True)
+    vp = np.array(v_pages, copy=True)
+    fp8 = kp.dtype == np.uint8
+    ks = np.array(k_scale, dtype=np.float32, copy=True) if fp8 else None
+    vs = np.array(v_scale, dtype=np.float32, copy=True) if fp8 else None
+    pt, ptp = _c(page_table, np.int32)
+    sl, slp = _c(seq_lens, np.int32)
+    kn, knp = _c(k_new, np.uint16)
+    vn, vnp = _c(v_new, np.uint16)
+    num_pages, Hk, P, D = kp.shape
+    lib().oracle_append_kv(kp.ctypes.data_as(_P), vp.ctypes.data_as(_P),
+                           ks.ctypes.data_as(_P) if fp8 else None,
+                           vs.ctypes.data_as(_P) if fp8 else None, 1 if fp8 else 0, ptp,
+                           pt.shape[1], slp, len(sl), Hk, D, P, knp, vnp)
+    return kp, vp, ks, vs
