@@ -1,7 +1,8 @@
 """Plant plausible mistakes in a COPY of the oracle source and check that a pin catches
-each one.  This shows the pins in test_oracle_pins.py constrain every step of the oracle
-(head map, page/slot indexing, scale, softmax, lse, split boundaries, merge, decoders,
-causal bound).  The real oracle source is never modified."""
+each one.  This shows the pins in test_oracle_pins.py and test_append_cpu.py constrain
+every step of the oracle (head map, page/slot indexing, scale, softmax, lse, split
+boundaries, merge, decoders, causal bound, KV append position, e4m3 encoding and the
+append scale).  The real oracle source is never modified."""
 import os
 import subprocess
 import tempfile
@@ -11,6 +12,7 @@ import pytest
 
 from oracle import build as obuild
 from oracle import oracle
+from tests import test_append_cpu as append_pins
 from tests import test_oracle_pins as pins
 
 MUTANTS = {
@@ -35,16 +37,23 @@ MUTANTS = {
                          "qd[d] = oracle_bf16_to_f64(q[((int64_t)b * Hq + j) * D + d]);"),
     "fp8_scale_ignored": ("* scale[phys * Hk + kvh];", ";"),
     "empty_split_weighed": ("if (lse_part[(int64_t)s * rows + r] == -INFINITY)\n                continue;", ""),
+    "append_slot_off_by_one": ("int slot = t % P;\n        for (int kvh", "int slot = (t + 1) % P;\n        for (int kvh"),
+    "append_at_L": ("int t = L - 1;\n        int64_t phys", "int t = L - 2 < 0 ? 0 : L - 2;\n        int64_t phys"),
+    "e4m3_ties_up": ("if (d < bd || (d == bd && (c & 1) == 0)) {", "if (d <= bd) {"),
+    "e4m3_inf_not_saturated": ("return (uint8_t)((sign << 7) | 0x7e);", "return 0x7f;"),
+    "append_scale_not_448": ("scale[si] = amax > 0.0f ? amax / 448.0f : 1.0f;",
+                             "scale[si] = amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    "append_keeps_no_scale": ("if (slot == 0) {\n                    float amax", "if (slot >= 0) {\n                    float amax"),
 }
 
 
 def _pins():
     """Every pin, as zero-argument callables (parametrized ones expanded)."""
     fns = []
-    for name in dir(pins):
+    for mod, name in [(m, n) for m in (pins, append_pins) for n in dir(m)]:
         if not name.startswith("test_"):
             continue
-        f = getattr(pins, name)
+        f = getattr(mod, name)
         marks = getattr(f, "pytestmark", [])
         params = [m for m in marks if m.name == "parametrize"]
         if not params:
