@@ -200,6 +200,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="decode workloads: launch the timed steps one by one from the host "
+                         "instead of replaying them as one captured CUDA graph")
     ap.add_argument("--append", action="store_true",
                     help="decode workloads: time gqa_paged_append_decode (each step first "
                          "writes the new token's K/V into its page)")
@@ -356,15 +359,16 @@ def main():
         v_new = torch.randn(B, Hk, D, generator=gk).to(torch.bfloat16).to(dev)
         launches += 1
 
-    def step():
+    def step(on=None):
+        on = stream if on is None else on
         if a.append:
             binding.gqa_paged_append_decode(q, k_new, v_new, kp, vp, pt, sl, case.scale,
                                             num_splits=S, pack_gqa=pack, k_scale=ks, v_scale=vs,
-                                            out=out, lse=lse, workspace=ws, stream=stream)
+                                            out=out, lse=lse, workspace=ws, stream=on)
             return
         binding.gqa_paged_decode(q, kp, vp, pt, sl, case.scale, num_splits=S, pack_gqa=pack,
                                  k_scale=ks, v_scale=vs, out=out, lse=lse, workspace=ws,
-                                 stream=stream)
+                                 stream=on)
 
     def barrier():
         if dist is not None:
@@ -379,17 +383,36 @@ def main():
 
     for _ in range(max(3, a.warmup)):
         step()
+    graph = None
+    if not a.eager:
+        # the timed steps, captured once: the replay launches them with no host work between
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for _ in range(a.steps):
+                    step(side)
+        stream.wait_stream(side)
+        graph.replay()  # warm replay
+        torch.cuda.synchronize(dev)
     barrier()
     clocks = ClockSampler(local)
     clocks.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     ev0.record(stream)
-    for _ in range(a.steps):
-        step()
+    if graph is not None:
+        graph.replay()
+    else:
+        for _ in range(a.steps):
+            step()
     ev1.record(stream)
     barrier()
     ms = ev0.elapsed_time(ev1) / a.steps
+    if graph is not None:
+        torch.cuda.synchronize(dev)
+        del graph
     clk = clocks.stop()
     ms = max_over_ranks(ms, dist, dev)
 
@@ -488,6 +511,7 @@ def main():
             "workload": workload_name(a),
             "B_per_gpu": B, "global_batch": B * world, "ctx": a.ctx, "Hq": Hq, "Hk": Hk,
             "head_dim": D, "page_size": P, "num_splits": S, "pack_gqa": pack,
+            "launch": "eager launches" if a.eager else "CUDA graph of the timed steps (captured once, replayed)",
             "schedule": ("balanced persistent (one launch)" if S == 0 and launches == 1 else
                          "balanced persistent + merge of cut units (two launches)" if S == 0 else
                          f"{S} splits + merge"),

@@ -250,6 +250,38 @@ def test_chained_decodes_read_the_previous_output():
               what=f"chained launch {i + 1}")
 
 
+@pytest.mark.parametrize("lens", [[64] * 64, [2048] * 2])
+def test_decode_replays_in_a_cuda_graph(lens):
+    """The balanced schedule captured in a CUDA graph (both merge variants: in-launch for
+    many short units, the separate merge kernel for two long sequences) replays to the
+    eager result, bit for bit."""
+    case = inputs.make_decode_case(len(lens), 32, 8, 128, 16, lens, seed=21)
+    d = to_dev(case)
+    B = len(lens)
+    ws = binding.new_workspace(binding.gqa_paged_decode_workspace_size(
+        B, 32, 8, 128, 16, d["pt"].shape[1] * 16, 0, 0), DEV)
+    out = torch.empty(B, 32, 128, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, 32, dtype=torch.float32, device=DEV)
+    binding.gqa_paged_decode(d["q"], d["k"], d["v"], d["pt"], d["sl"], case.scale, out=out,
+                             lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    eager_o, eager_l = out.clone(), lse.clone()
+    out.zero_()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+        for _ in range(2):
+            binding.gqa_paged_decode(d["q"], d["k"], d["v"], d["pt"], d["sl"], case.scale,
+                                     out=out, lse=lse, workspace=ws, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize()
+    assert binding.gqa_get_error(ws) == 0
+    assert torch.equal(out, eager_o) and torch.equal(lse, eager_l)
+    del g
+
+
 @pytest.mark.parametrize("lens", [[1], [2048], [16] * 37, [0, 0, 5], [3000, 1, 17, 0, 900, 4096]])
 def test_balanced_schedule_shapes(lens):
     """The balanced persistent schedule (num_splits = 0) on batch shapes whose units are
