@@ -630,6 +630,17 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 // merging pieces) never holds up the other warps' streams.
 
 constexpr int kMinTilesPerWorker = 16;
+// When one worker per kMinTilesPerWorker tiles would leave more than three quarters of the
+// workers idle (a few short sequences), one per kMinTilesPerWorkerSmall tiles: such
+// streams are latency-bound, so more of them in flight finish sooner.
+constexpr int kMinTilesPerWorkerSmall = 4;
+
+// Workers of a launch with T tiles and `workers` consumer warps.
+__device__ __forceinline__ long long sk_workers(long long T, long long workers) {
+    const long long nw = T / kMinTilesPerWorker;
+    const long long per = nw * 4 < workers ? kMinTilesPerWorkerSmall : kMinTilesPerWorker;
+    return min(workers, max(1LL, T / per));
+}
 // Launches whose units average more than kDeferMinWorkersPerUnit workers each leave their
 // pieces to a second kernel (piece_merge_kernel, the DEFER instance), which merges every
 // cut unit in parallel; otherwise the last piece of a unit to finish merges all of them in
@@ -808,8 +819,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     __syncthreads();
 
     const long long T = (long long)U * pre[B];
-    const long long NW = min((long long)gridDim.x * kConsumerWarps,
-                             max(1LL, T / kMinTilesPerWorker));
+    const long long NW = sk_workers(T, (long long)gridDim.x * kConsumerWarps);
     const long long W0cta = (long long)blockIdx.x * kConsumerWarps;
 
     // Sequences with no tokens have no tiles: their outputs are written here (zeros, -inf).
@@ -1052,7 +1062,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
     if (warp == 0) tile_prefix<TT>(a, pre_m, a.pt_stride * a.P, nullptr, lane);
     __syncthreads();
     const long long T = (long long)U * pre_m[a.B];
-    const long long NW = min((long long)a.grid * kConsumerWarps, max(1LL, T / kMinTilesPerWorker));
+    const long long NW = sk_workers(T, (long long)a.grid * kConsumerWarps);
     const int slot_floats = (heads_per_cta * (D + 1) + 3) & ~3;
     for (long long u = blockIdx.x; u < (long long)a.B * U; u += gridDim.x) {
         const int b = (int)(u / U), y = (int)(u % U);

@@ -1,7 +1,8 @@
 """Host check of the balanced persistent decode schedule's integer arithmetic: the tile
 partition among workers, the owner of a tile, and the merge pieces of units that workers
 share.  The formulas are the ones decode_sk_kernel evaluates (restated here): worker W
-owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // 16)); the owner
+owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // per)), per = 16
+tiles, or 4 when T // 16 workers would be under a quarter of them; the owner
 of tile t is ((t+1)*NW + T-1)//T - 1;
 a unit cut between workers leaves one piece per worker, side 1 for the worker where the
 unit begins and side 0 for the others.  The last piece of a unit merges them in the same
@@ -14,7 +15,8 @@ import pytest
 
 
 def n_workers(workers, T):
-    return min(workers, max(1, T // 16))
+    per = 4 if (T // 16) * 4 < workers else 16
+    return min(workers, max(1, T // per))
 
 
 def start(W, T, NW):
@@ -64,7 +66,8 @@ def test_partition_and_owner(workers):
             cover += list(range(start(W, T, NW), start(W + 1, T, NW)))
         assert cover == list(range(T))
         sizes = [start(W + 1, T, NW) - start(W, T, NW) for W in range(NW)]
-        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= min(16, T)
+        per = 4 if (T // 16) * 4 < workers else 16
+        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= min(per, T)
         for t in range(T):
             W = owner(t, T, NW)
             assert start(W, T, NW) <= t < start(W + 1, T, NW)
