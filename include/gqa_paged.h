@@ -36,8 +36,8 @@
  *     clears it.
  *   - Layouts are row-major (C order).  KV pools are [num_pages][Hk][page_size][head_dim]
  *     ("HND": each (page, kv head) block is one contiguous run).  q and out are bf16.
- *   - Sequence lengths count the current token(s): the caller has already written the
- *     new K/V into the cache.  The library never writes the cache.
+ *   - Sequence lengths count the current token(s): the new K/V are in the cache, written
+ *     by the caller or by gqa_paged_append_kv().  No other call writes the cache.
  *   - Page-table entries at or beyond ceil(seq_len / page_size) are never read; entries
  *     may repeat across and within sequences (shared prefix pages).
  *   - A sequence of length 0 yields output 0 and lse = -inf.
