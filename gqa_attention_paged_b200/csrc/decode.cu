@@ -621,9 +621,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 //
 // Flat tile space: sequence b owns tiles [U*pre[b], U*pre[b+1]) with pre[] the prefix of
 // nt_b = ceil(L_b / 16) and U = Hk * head chunks units per sequence; unit y of sequence
-// b owns [U*pre[b] + y*nt_b, ... + nt_b).  With T tiles and NW workers (at most one per
-// kMinTilesPerWorker tiles), worker W owns [W*T/NW, (W+1)*T/NW) (floor divisions): every
-// worker gets one tile more or less than any other.
+// b owns [U*pre[b] + y*nt_b, ... + nt_b).  With T tiles and NW workers (sk_workers: at most
+// one per kMinTilesPerWorker tiles, or per kMinTilesPerWorkerSmall for small launches),
+// worker W owns [W*T/NW, (W+1)*T/NW) (floor divisions): every worker gets one tile more or
+// less than any other.
 //
 // Each consumer warp is one worker with a private sub-ring of S/4 stages fed by its own
 // producer lane (lane w of warp 4), so a warp that pauses (loading the next unit's q,
