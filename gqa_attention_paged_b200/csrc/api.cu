@@ -393,6 +393,9 @@ int gqa_paged_append_decode(const void *q, const void *k_new, const void *v_new,
     if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
     if (kv_dtype == GQA_KV_FP8_E4M3 && head_dim != 128) return GQA_ERR_DTYPE;
     if (!workspace || !aligned(workspace, 256)) return workspace ? GQA_ERR_WORKSPACE : GQA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+        (lse && !aligned(lse, 4)))
+        return GQA_ERR_ALIGN;
     const bool sk = use_stream_k(num_splits, B);
     const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
     if (workspace_bytes < gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,

@@ -86,6 +86,27 @@ def test_decode_rejects_bad_arguments_on_the_host(kw, status):
     assert _decode(**kw) == status
 
 
+def _append_decode(**kw):
+    args = dict(q=_fake(), kn=_fake(), vn=_fake(), k=_fake(), v=_fake(), ks=None, vs=None,
+                kvd=0, pt=_fake(), pts=8, sl=_fake(), B=2, Hq=8, Hk=2, D=64, P=16, npg=16,
+                scale=0.125, S=0, pack=1, out=_fake(), lse=None, ws=_fake(), wsb=1 << 26,
+                st=None)
+    args.update(kw)
+    return binding.load().gqa_paged_append_decode(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), -1), (dict(kn=None), -1), (dict(ws=None), -1),
+    (dict(Hq=6, Hk=4), -2), (dict(D=96), -2), (dict(P=8), -2), (dict(B=-1), -2),
+    (dict(kvd=1), -3), (dict(S=65), -4), (dict(wsb=16), -5),
+    (dict(q=_fake(0x10008)), -9), (dict(out=_fake(0x10004)), -9), (dict(k=_fake(0x10002)), -9),
+])
+def test_append_decode_rejects_before_writing(kw, status):
+    """Every rejection happens on the host before the append kernel is enqueued (these
+    pointers are never dereferenced), so a rejected call leaves the cache untouched."""
+    assert _append_decode(**kw) == status
+
+
 def test_host_helpers():
     lib = binding.load()
     assert lib.gqa_paged_decode_workspace_size(4, 8, 2, 64, 16, 256, 0, 1) == 256
