@@ -1,12 +1,16 @@
 """Benchmark: paged GQA decode on B200 -- HBM GB/s (% of peak) and queries/s at B=64, 2K ctx.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--B 64] [--ctx 2048] [--splits 0] [--no-pack] [--kv bf16|fp8_e4m3]
+                    [--workload decode|long70b|prefill] [--B 64] [--ctx 2048] [--splits 0]
+                    [--no-pack] [--kv bf16|fp8_e4m3] [--append] [--eager] [--no-secondary]
 
-One step = one gqa_paged_decode call (decode kernel + log-sum-exp merge when split) over
-a batch of B sequences, each with `ctx` tokens of paged history (Hq=32, Hk=8, D=128,
-page_size=16, seeded synthetic N(0,1) data).  Under torchrun every rank runs its own batch
-(weak scaling; no collective on the data path) and rank 0 prints one JSON line.
+One step = one gqa_paged_decode call (the balanced decode kernel, plus the merge kernel
+when the call merges separately) over a batch of B sequences, each with `ctx` tokens of
+paged history (Hq=32, Hk=8, D=128, page_size=16, seeded synthetic N(0,1) data).  Under
+torchrun every rank runs its own batch (weak scaling; no collective on the data path) and
+rank 0 prints one JSON line.  With no flags, the line also carries a `secondary` list: the
+causal chunked prefill (TFLOP/s) and the 70B-shaped long-context decode with e4m3 KV
+(GB/s), each measured the same way in the same run.
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -25,9 +29,10 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "GQA paged decode: HBM GB/s (% of B200 peak) and queries/s at B=64, 2K ctx"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
-# ------------------------------------------------------------------------ byte model
+# ------------------------------------------------------------------------ byte / flop model
 
 def decode_kv_bytes(seq_lens, Hk, D, elem):
     """Algorithmic K+V bytes of one decode step: every valid token's K and V row of every
@@ -43,6 +48,13 @@ def decode_step_bytes(seq_lens, Hq, Hk, D, elem, P=16):
     if elem == 1:
         b += 2 * 4 * Hk * sum((int(L) + P - 1) // P for L in seq_lens)
     return b
+
+
+def prefill_flops(prior_lens, q_lens, Hq, D):
+    """4*Hq*D per unmasked (query, key) pair: row i of a chunk of Lq after `prior` keys
+    sees prior + i + 1 keys."""
+    pairs = sum(int(Lq) * int(p) + int(Lq) * (int(Lq) + 1) // 2 for p, Lq in zip(prior_lens, q_lens))
+    return 4 * Hq * D * pairs
 
 
 def rank_seed(seed, rank):
@@ -66,14 +78,36 @@ def aggregate_gbs(step_bytes_per_rank, world, ms_max):
     return world * step_bytes_per_rank / (ms_max * 1e-3) / 1e9
 
 
-def peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def spread(ms_list):
+    """median / min / p90 of per-step times (ms); None when nothing was repeated."""
+    if not ms_list:
+        return None
+    s = sorted(ms_list)
+    p90 = s[min(len(s) - 1, int(math.ceil(0.9 * len(s))) - 1)]
+    return {"median_ms": round(statistics.median(s), 5), "min_ms": round(s[0], 5),
+            "p90_ms": round(p90, 5), "samples": len(s)}
+
+
+def _peaks_file():
     try:
-        with open(path) as f:
-            p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return None
+
+
+def peaks():
+    p = _peaks_file()
+    if p and "hbm_gbs" in p:
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    p = _peaks_file()
+    if p and "bf16_tflops" in p:
+        return float(p["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_src_sha():
@@ -86,7 +120,7 @@ def kernel_src_sha():
 
 
 def traffic_from_profile(workload_key):
-    """DRAM bytes per decode launch from the committed ncu summary, or None if absent or
+    """DRAM bytes per decode call from the committed ncu summary, or None if absent or
     taken on a different kernel source."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
@@ -118,7 +152,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -132,7 +166,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
+        sm, mx, power, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
@@ -142,6 +176,7 @@ class ClockSampler:
                 try:
                     sm.append(float(parts[1]))
                     mx = float(parts[2])
+                    power.append(float(parts[3]))
                 except ValueError:
                     continue
                 for n, v in zip(names, parts[5:9]):
@@ -150,26 +185,145 @@ class ClockSampler:
         os.unlink(self.path)
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        # samples under load: power well above idle
+        loaded = [s for s, p in zip(sm, power) if p > 250.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "samples_under_load": len([p for p in power if p > 250.0])}
 
 
-# ------------------------------------------------------------------------ CPU oracle leg
+# ------------------------------------------------------------------------ timing helpers
+
+def timed_graph(step, K, stream, dev, repeat_s=1.0):
+    """Capture K steps as one CUDA graph and time its replay with CUDA events on `stream`:
+    the contract timing (one replay, exactly K steps), then further replays for about
+    `repeat_s` seconds, whose per-step times give median / min / p90."""
+    import torch
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(K):
+                step(side)
+    stream.wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / K
+    per = []
+    t_end = time.perf_counter() + repeat_s
+    while time.perf_counter() < t_end and len(per) < 2000:
+        evs = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        per += [a.elapsed_time(b) / K for a, b in evs]
+    del graph
+    torch.cuda.synchronize(dev)
+    return ms, spread(per)
+
+
+def timed_eager(step, K, stream, dev, repeat_s=1.0):
+    """Launch K steps one by one from the host between one pair of CUDA events, then
+    repeat for about `repeat_s` seconds for median / min / p90."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K):
+        step(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / K
+    per = []
+    t_end = time.perf_counter() + repeat_s
+    while time.perf_counter() < t_end and len(per) < 200:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            step(stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        per.append(a.elapsed_time(b) / K)
+    return ms, spread(per)
+
+
+def e2e_pipelined(dev, stream, h_in, d_in, d_out, h_out, run, steps):
+    """End-to-end time per step through the public API, as a serving loop would issue it:
+    step i's inputs are copied from pinned host memory into one of two device input sets on
+    a copy stream while step i-1 computes; the compute of step i (run(slot, stream)) waits
+    for them; its results are copied back to one of two pinned host sets on a third stream
+    while step i+1 computes.  Every step's copies are inside the timed region.
+
+    h_in: pinned host tensors; d_in: per input, a pair of device buffers; d_out: per
+    output, a pair of device buffers; h_out: per output, a pair of pinned host buffers."""
+    import torch
+    cp, dh = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+    copied_out = [torch.cuda.Event() for _ in range(2)]
+
+    def one(i):
+        s = i % 2
+        if i >= 2:
+            cp.wait_event(consumed[s])       # step i-2 has read this input set
+        with torch.cuda.stream(cp):
+            for h, d in zip(h_in, d_in):
+                d[s].copy_(h, non_blocking=True)
+        in_ready[s].record(cp)
+        stream.wait_event(in_ready[s])
+        if i >= 2:
+            stream.wait_event(copied_out[s])  # step i-2's results have left this output set
+        run(s, stream)
+        consumed[s].record(stream)
+        dh.wait_event(consumed[s])
+        with torch.cuda.stream(dh):
+            for d, h in zip(d_out, h_out):
+                h[s].copy_(d[s], non_blocking=True)
+        copied_out[s].record(dh)
+
+    for i in range(4):  # warm
+        one(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    cp.wait_event(e0)
+    dh.wait_event(e0)
+    for i in range(steps):
+        one(i)
+    stream.wait_stream(dh)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / steps
+
+
+# ------------------------------------------------------------------------ CPU oracle legs
+
+def _bits(t):
+    import numpy as np
+    import torch
+    t = t.contiguous()
+    return t.view(torch.int16).numpy().view(np.uint16) if t.dtype.itemsize == 2 \
+        else t.view(torch.uint8).numpy()
+
 
 def run_oracle_sample(case, rows, min_seconds):
     """Time the fp64 oracle on sequences `rows` of `case`, repeating until min_seconds."""
-    import numpy as np
     from oracle import oracle
 
     kv = case.kv
-
-    def bits(t):
-        t = t.contiguous()
-        return t.view(__import__("torch").int16).numpy().view(np.uint16) if t.dtype.itemsize == 2 \
-            else t.view(__import__("torch").uint8).numpy()
-
-    q = bits(case.q[rows])
-    kp, vp = bits(kv.k_pages), bits(kv.v_pages)
+    q = _bits(case.q[rows])
+    kp, vp = _bits(kv.k_pages), _bits(kv.v_pages)
     pt = kv.page_table[rows].numpy()
     sl = kv.seq_lens[rows].numpy()
     ks = None if kv.k_scale is None else kv.k_scale.numpy()
@@ -184,9 +338,40 @@ def run_oracle_sample(case, rows, min_seconds):
     return el / reps, reps, oracle.num_threads()
 
 
-# ------------------------------------------------------------------------ main
+def run_oracle_prefill_sample(case, rows_per_seq, min_seconds):
+    """Time the fp64 oracle on the last `rows_per_seq` query rows of every chunk (same
+    positions and keys as in the full chunk).  Returns (seconds per pass, flops of the
+    sample, repeats, threads)."""
+    import numpy as np
+    from oracle import oracle
 
-def parse():
+    kv = case.kv
+    cu = case.cu_q.tolist()
+    lens = kv.seq_lens.tolist()
+    idx, cu_s, prior, qls = [], [0], [], []
+    for b in range(len(lens)):
+        n = min(rows_per_seq, cu[b + 1] - cu[b])
+        idx += list(range(cu[b + 1] - n, cu[b + 1]))
+        cu_s.append(cu_s[-1] + n)
+        prior.append(lens[b] - n)
+        qls.append(n)
+    q = _bits(case.q[idx])
+    kp, vp = _bits(kv.k_pages), _bits(kv.v_pages)
+    pt, sl = kv.page_table.numpy(), kv.seq_lens.numpy()
+    cu_np = np.array(cu_s, np.int32)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.prefill(q, cu_np, kp, vp, pt, sl, case.scale, True)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return el / reps, prefill_flops(prior, qls, case.Hq, case.head_dim), reps, oracle.num_threads()
+
+
+# ------------------------------------------------------------------------ arguments
+
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -200,6 +385,10 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="headline run: skip the prefill and e4m3 long-context lines")
+    ap.add_argument("--repeat-seconds", type=float, default=1.0,
+                    help="seconds of repeated replays behind median / min / p90")
     ap.add_argument("--eager", action="store_true",
                     help="decode workloads: launch the timed steps one by one from the host "
                          "instead of replaying them as one captured CUDA graph")
@@ -210,7 +399,25 @@ def parse():
                     help="decode: the headline (paged GQA decode); prefill: causal chunked "
                          "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]; "
                          "long70b: B=4 decode at 8K/16K/24K/32K, Hq=64 Hk=8, page 64 (--kv)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def decode_metric(a):
+    """The metric string of a decode line: the headline's at B=64 / 2K with bf16 KV, and a
+    string naming the workload everywhere else."""
+    kv = "" if a.kv == "bf16" else ", e4m3 KV"
+    what = "GQA paged KV append + decode" if a.append else "GQA paged decode"
+    if a.workload == "long70b":
+        return (f"{what}, 70B-shaped long context (B=4, ctx 8K-32K, Hq=64 Hk=8{kv}): "
+                "HBM GB/s (% of B200 peak)")
+    if not a.append and a.kv == "bf16" and a.B == 64 and a.ctx == 2048:
+        return METRIC
+    ctx = f"{a.ctx // 1024}K" if a.ctx % 1024 == 0 else str(a.ctx)
+    return f"{what}: HBM GB/s (% of B200 peak) and queries/s at B={a.B}, {ctx} ctx{kv}"
+
+
+PREFILL_METRIC = ("causal chunked prefill over a paged KV cache (B=8, 512-token chunks, "
+                  "prior ~ U[0,4096]): TFLOP/s of unmasked pairs (% of bf16 peak)")
 
 
 def workload_name(a):
@@ -220,28 +427,12 @@ def workload_name(a):
             f"Hk=8 D=128 page_size=16 kv={a.kv}")
 
 
-def prefill_flops(prior_lens, q_lens, Hq, D):
-    """4*Hq*D per unmasked (query, key) pair: row i of a chunk of Lq after `prior` keys
-    sees prior + i + 1 keys."""
-    pairs = sum(int(Lq) * int(p) + int(Lq) * (int(Lq) + 1) // 2 for p, Lq in zip(prior_lens, q_lens))
-    return 4 * Hq * D * pairs
+# ------------------------------------------------------------------------ prefill
 
-
-def tensor_peak():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    try:
-        with open(path) as f:
-            p = json.load(f)
-        return float(p["bf16_tflops"]), "measured"
-    except Exception:
-        return 1590.0, "fallback"
-
-
-def run_prefill_bench(a):
+def measure_prefill(a, dev, with_cpu):
     import torch
     from gqa_attention_paged_b200 import binding, inputs
 
-    dev = torch.device("cuda", 0)
     case = inputs.chunked_prefill(seed=a.seed)
     kv = case.kv
     q, cu = case.q.to(dev), case.cu_q.to(dev)
@@ -252,9 +443,12 @@ def run_prefill_bench(a):
     ws = binding.new_workspace(binding.gqa_paged_prefill_workspace_size(T, Hq, D), dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        binding.gqa_paged_prefill(q, cu, kp, vp, pt, sl, case.scale, case.max_q_len, out=out,
-                                  lse=lse, workspace=ws, stream=stream)
+    def step(on=None, qq=None, cc=None, ptt=None, sll=None, oo=None, ll=None):
+        binding.gqa_paged_prefill(q if qq is None else qq, cu if cc is None else cc, kp, vp,
+                                  pt if ptt is None else ptt, sl if sll is None else sll,
+                                  case.scale, case.max_q_len, out=out if oo is None else oo,
+                                  lse=lse if ll is None else ll, workspace=ws,
+                                  stream=stream if on is None else on)
 
     step()
     torch.cuda.synchronize(dev)
@@ -265,67 +459,90 @@ def run_prefill_bench(a):
     # The step's K/V (84 MB) fit in L2, so L2 is flushed before every timed step by
     # writing a buffer twice its size; only the launch itself is inside the events.
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    clocks = ClockSampler(0)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(a.steps)]
-    for e0, e1 in ev:
-        flush.fill_(1)
-        e0.record(stream)
-        step()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / a.steps
+
+    def timed(n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for e0, e1 in ev:
+            flush.fill_(1)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    per = timed(a.steps)
+    ms = sum(per) / a.steps
+    more, t_end = [], time.perf_counter() + a.repeat_seconds
+    while time.perf_counter() < t_end and len(more) < 2000:
+        more += timed(20)
     clk = clocks.stop()
+
+    # end to end: q, cu_q, page table and seq_lens H2D from pinned memory, out and lse D2H
+    # (the paged K/V, the chunk's included, are device-resident: written by the layers
+    # that project them)
+    hin = [case.q.pin_memory(), case.cu_q.pin_memory(), kv.page_table.pin_memory(),
+           kv.seq_lens.pin_memory()]
+    din = [(x.to(dev), x.to(dev)) for x in hin]
+    dout = [(out, torch.empty_like(out)), (lse, torch.empty_like(lse))]
+    hout = [(torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+             torch.empty(out.shape, dtype=out.dtype).pin_memory()),
+            (torch.empty(lse.shape).pin_memory(), torch.empty(lse.shape).pin_memory())]
+
+    def run(s, on):
+        step(on, din[0][s], din[1][s], din[2][s], din[3][s], dout[0][s], dout[1][s])
+
+    e2e_ms = e2e_pipelined(dev, stream, hin, din, dout, hout, run, a.steps)
+    h2d = sum(x.numel() * x.element_size() for x in hin)
+    d2h = sum(p[0].numel() * p[0].element_size() for p in hout)
+
     q_lens = (case.cu_q[1:] - case.cu_q[:-1]).tolist()
     prior = [int(L) - int(x) for L, x in zip(kv.seq_lens.tolist(), q_lens)]
     flops = prefill_flops(prior, q_lens, Hq, D)
     tf = flops / (ms * 1e-3) / 1e12
     peak, kind = tensor_peak()
-    print(json.dumps({
-        "metric": "causal chunked prefill over a paged KV cache: TFLOP/s (unmasked pairs)",
-        "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps,
-        "warmup": max(3, a.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True,
+    cpu = None
+    if with_cpu:
+        sec, sflops, reps, cores = run_oracle_prefill_sample(case, 4, min(a.cpu_seconds, 8.0))
+        cpu = {"value": round(sflops / sec / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+               "kind": "oracle",
+               "sample": f"the last 4 query rows of each of the 8 chunks (same keys and "
+                         f"positions as in the full chunk), {reps} repeats, "
+                         f"{sec * reps:.1f} s of CPU work; TFLOP/s of the same flop model"}
+    return {
+        "metric": PREFILL_METRIC,
+        "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+        "steps": a.steps, "warmup": max(3, a.warmup), "higher_is_better": True,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v)",
         "config": {"workload": "chunked prefill B=8 Lq=512 prior~U[0,4096] Hq=32 Hk=8 D=128 P=16",
                    "flops_per_step": flops, "prior_lens": prior,
                    "l2": "flushed before every timed step (256 MB write outside the events)"},
+        "pct_of_bf16_peak": round(100 * tf / peak, 2),
         "tokens_per_s": round(sum(q_lens) / (ms * 1e-3), 1),
+        "spread": spread(more) if more else None,
         "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(tf / peak, 4), "traffic": None,
-                     "peak_source": f"{kind} (bf16_tflops, burst cuBLAS GEMM)"},
+                     "peak_source": f"{kind} (bf16_tflops, burst cuBLAS GEMM)",
+                     "kernel": "prefill_kernel (plan kernel included in the step time)"},
+        "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 5),
+                "note": "q, cu_q, page table, seq_lens H2D from pinned memory on a copy stream, "
+                        "out+lse D2H on a third stream, double-buffered so step i's copies "
+                        "overlap steps i-1 / i+1; eager gqa_paged_prefill calls; L2 not flushed"},
         "gpu_launches": 2 * a.steps,  # the plan kernel and the prefill kernel per step
-        "clocks": clk}))
-    return 0
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
 
 
-def main():
-    a = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+# ------------------------------------------------------------------------ decode
 
-    if a.workload == "prefill" and a.impl == "ours":
-        return run_prefill_bench(a)
-    if a.impl == "reference":
-        if rank != 0:
-            return 0
-        return reference_arm(a, world)
-
+def measure_decode(a, dev, rank, world, dist, with_cpu):
     import torch
     from gqa_attention_paged_b200 import binding, inputs
-
-    if not torch.cuda.is_available():
-        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
-        return 1
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
 
     if a.workload == "long70b":
         case = inputs.long70b_decode(seed=rank_seed(a.seed, rank), kv_dtype=a.kv)
@@ -359,23 +576,27 @@ def main():
         v_new = torch.randn(B, Hk, D, generator=gk).to(torch.bfloat16).to(dev)
         launches += 1
 
-    def step(on=None):
+    def step(on=None, qq=None, ptt=None, sll=None, oo=None, ll=None):
         on = stream if on is None else on
+        qq = q if qq is None else qq
+        ptt = pt if ptt is None else ptt
+        sll = sl if sll is None else sll
+        oo = out if oo is None else oo
+        ll = lse if ll is None else ll
         if a.append:
-            binding.gqa_paged_append_decode(q, k_new, v_new, kp, vp, pt, sl, case.scale,
+            binding.gqa_paged_append_decode(qq, k_new, v_new, kp, vp, ptt, sll, case.scale,
                                             num_splits=S, pack_gqa=pack, k_scale=ks, v_scale=vs,
-                                            out=out, lse=lse, workspace=ws, stream=on)
+                                            out=oo, lse=ll, workspace=ws, stream=on)
             return
-        binding.gqa_paged_decode(q, kp, vp, pt, sl, case.scale, num_splits=S, pack_gqa=pack,
-                                 k_scale=ks, v_scale=vs, out=out, lse=lse, workspace=ws,
-                                 stream=on)
+        binding.gqa_paged_decode(qq, kp, vp, ptt, sll, case.scale, num_splits=S, pack_gqa=pack,
+                                 k_scale=ks, v_scale=vs, out=oo, lse=ll, workspace=ws, stream=on)
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # parity spot check of this exact launch configuration before timing
+    # sanity check of this exact launch configuration before timing
     step()
     torch.cuda.synchronize(dev)
     assert binding.gqa_get_error(ws) == 0
@@ -383,36 +604,15 @@ def main():
 
     for _ in range(max(3, a.warmup)):
         step()
-    graph = None
-    if not a.eager:
-        # the timed steps, captured once: the replay launches them with no host work between
-        graph = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(graph, stream=side):
-                for _ in range(a.steps):
-                    step(side)
-        stream.wait_stream(side)
-        graph.replay()  # warm replay
-        torch.cuda.synchronize(dev)
     barrier()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
-    ev0.record(stream)
-    if graph is not None:
-        graph.replay()
+    if a.eager:
+        ms, sp = timed_eager(step, a.steps, stream, dev, a.repeat_seconds)
     else:
-        for _ in range(a.steps):
-            step()
-    ev1.record(stream)
+        ms, sp = timed_graph(step, a.steps, stream, dev, a.repeat_seconds)
     barrier()
-    ms = ev0.elapsed_time(ev1) / a.steps
-    if graph is not None:
-        torch.cuda.synchronize(dev)
-        del graph
     clk = clocks.stop()
     ms = max_over_ranks(ms, dist, dev)
 
@@ -441,33 +641,22 @@ def main():
 
     # end to end through the public API: per step, the step's inputs (q, page table,
     # sequence lengths) copied from pinned host memory, the decode, and the result (out,
-    # lse) copied back; the KV cache is device-resident state.
-    hq = case.q.pin_memory()
-    hpt = kv.page_table.pin_memory()
-    hsl = kv.seq_lens.pin_memory()
-    hout = torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory()
-    hlse = torch.empty(B, Hq, dtype=torch.float32).pin_memory()
-    h2d = hq.numel() * 2 + hpt.numel() * 4 + hsl.numel() * 4
-    d2h = hout.numel() * 2 + hlse.numel() * 4
+    # lse) copied back; the KV cache is device-resident state.  Pipelined as a serving
+    # loop issues it (see e2e_pipelined).
+    hin = [case.q.pin_memory(), kv.page_table.pin_memory(), kv.seq_lens.pin_memory()]
+    din = [(q, q.clone()), (pt, pt.clone()), (sl, sl.clone())]
+    dout = [(out, torch.empty_like(out)), (lse, torch.empty_like(lse))]
+    hout = [(torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory()),
+            (torch.empty(B, Hq).pin_memory(), torch.empty(B, Hq).pin_memory())]
+    h2d = sum(x.numel() * x.element_size() for x in hin)
+    d2h = sum(p[0].numel() * p[0].element_size() for p in hout)
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        pt.copy_(hpt, non_blocking=True)
-        sl.copy_(hsl, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+    def run(s, on):
+        step(on, din[0][s], din[1][s], din[2][s], dout[0][s], dout[1][s])
 
-    for _ in range(3):
-        e2e_step()
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(a.steps):
-        e2e_step()
-    e1.record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dist, dev)
+    e2e_ms = max_over_ranks(e2e_pipelined(dev, stream, hin, din, dout, hout, run, a.steps), dist, dev)
 
     lens = [int(x) for x in kv.seq_lens]
     step_bytes = decode_step_bytes(lens, Hq, Hk, D, elem, P)
@@ -477,11 +666,12 @@ def main():
     gbs = aggregate_gbs(step_bytes, world, ms)
     kern_gbs = step_bytes / (kern_ms * 1e-3) / 1e9
     e2e_gbs = aggregate_gbs(step_bytes, world, e2e_ms)
-    wkey = f"B{B}_ctx{a.ctx}_{a.kv}_S{S}_pack{int(pack)}"
-    traffic = traffic_from_profile(wkey)
+    wkey = (f"long70b_{a.kv}_S{S}_pack{int(pack)}" if a.workload == "long70b"
+            else f"B{B}_ctx{a.ctx}_{a.kv}_S{S}_pack{int(pack)}")
+    traffic = None if a.append else traffic_from_profile(wkey)
 
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if with_cpu and rank == 0 and world == 1:
         rows = list(range(min(B, 8)))
         sec, reps, cores = run_oracle_sample(case, rows, a.cpu_seconds)
         sb = decode_step_bytes([lens[r] for r in rows], Hq, Hk, D, elem, P)
@@ -489,13 +679,8 @@ def main():
                "sample": f"{len(rows)} of {B} sequences (ctx {a.ctx}), {reps} repeats, "
                          f"{sec * reps:.1f} s of CPU work; GB/s of the same byte model"}
 
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return 0
-    line = {
-        "metric": METRIC,
+    return {
+        "metric": decode_metric(a),
         "value": round(gbs, 2),
         "unit": "GB/s",
         "n_gpus": world,
@@ -523,6 +708,7 @@ def main():
         "pct_of_hbm_peak": round(100 * gbs / world / peak, 2),
         "queries_per_s": round(world * B / (ms * 1e-3), 1),
         "head_queries_per_s": round(world * B * Hq / (ms * 1e-3), 1),
+        "spread": sp,
         "roofline": {"bound": "hbm", "achieved": round(kern_gbs, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(kern_gbs / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
@@ -530,15 +716,79 @@ def main():
                      "kernel": ("decode_sk_kernel (the whole call: one launch)" if S == 0 and launches == 1 else
                                 "decode_sk_kernel + piece_merge_kernel (the whole call)" if S == 0 else
                                 "decode_kernel (call time minus the separately timed lse_combine)"),
-                     "kernel_ms": round(kern_ms, 5), "combine_ms": round(comb_ms, 5)},
+                     "kernel_ms": round(kern_ms, 5), "combine_ms": round(comb_ms, 5),
+                     "traffic_key": wkey},
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
-                "note": "q, page table and seq_lens H2D from pinned memory, out+lse D2H, "
-                        "KV cache device-resident"},
+                "frac_of_device": round(ms / e2e_ms, 4),
+                "note": "q, page table and seq_lens H2D from pinned memory on a copy stream, "
+                        "out+lse D2H on a third stream, double-buffered so step i's copies "
+                        "overlap steps i-1 / i+1; eager gqa_paged_decode calls; KV cache "
+                        "device-resident"},
         "gpu_launches": a.steps * launches,
         "clocks": clk,
         "cpu_baseline": cpu,
     }
+
+
+def _secondary_summary(line):
+    keep = ("metric", "value", "unit", "ms_per_step", "spread", "roofline", "clocks", "e2e",
+            "cpu_baseline", "gpu_launches", "pct_of_hbm_peak", "pct_of_bf16_peak", "dtype")
+    s = {k: line[k] for k in keep if k in line}
+    s["workload"] = line["config"]["workload"]
+    return s
+
+
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        return reference_arm(a, world)
+
+    import torch
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    if a.workload == "prefill":
+        if rank != 0:
+            return 0
+        line = measure_prefill(a, dev, with_cpu=not a.no_cpu_baseline)
+        line.update({"n_gpus": 1, "scaling": "weak", "vs_baseline": None})
+        print(json.dumps(line))
+        return 0
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    headline = (a.workload == "decode" and not a.append and a.kv == "bf16" and a.B == 64
+                and a.ctx == 2048 and a.splits == 0 and not a.no_pack)
+    line = measure_decode(a, dev, rank, world, dist, with_cpu=not a.no_cpu_baseline)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    if headline and world == 1 and not a.no_secondary:
+        sec = []
+        pa = parse(["--steps", str(a.steps), "--warmup", str(a.warmup), "--workload", "prefill",
+                    "--repeat-seconds", str(a.repeat_seconds), "--cpu-seconds", str(a.cpu_seconds)])
+        sec.append(_secondary_summary(measure_prefill(pa, dev, with_cpu=not a.no_cpu_baseline)))
+        la = parse(["--steps", str(a.steps), "--warmup", str(a.warmup), "--workload", "long70b",
+                    "--kv", "fp8_e4m3", "--repeat-seconds", str(a.repeat_seconds)])
+        sec.append(_secondary_summary(measure_decode(la, dev, 0, 1, None, with_cpu=False)))
+        line["secondary"] = sec
     print(json.dumps(line))
     return 0
 
@@ -565,12 +815,13 @@ def reference_arm(a, world):
     v = sb / sec / 1e9
     line = {
         "impl": "reference",
-        "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "metric": decode_metric(a), "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(sec * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded inputs as the GPU arm)",
         "config": {"workload": workload_name(a), "B_per_gpu": a.B, "ctx": a.ctx,
                    "sample": f"{len(rows)} of {a.B} sequences per step"},
+        "spread": spread([s * 1e3 for s in per_step]),
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": f"{len(rows)} of {a.B} sequences per step, {a.steps} steps"},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
