@@ -34,6 +34,8 @@ SIGNATURES = {
     "gqa_pick_splits": (_I, [_I, _I, _I, _I, _I]),
     "gqa_paged_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                               ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
+    "gqa_paged_decode_partial": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                      ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
     "gqa_paged_decode_static_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
                                              _I, _I, _I, ctypes.c_float, _I, _I, _P, _P, _P]),
     "gqa_paged_prefill_workspace_size": (_SZ, [_I, _I, _I]),
@@ -192,6 +194,55 @@ def gqa_paged_decode(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tens
         workspace.numel(), _stream(stream))
     _check("gqa_paged_decode", st)
     return out, lse
+
+
+def gqa_paged_decode_partial(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                             page_table: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                             num_splits: int = 0, pack_gqa: bool = True,
+                             k_scale: Optional[torch.Tensor] = None,
+                             v_scale: Optional[torch.Tensor] = None,
+                             o_part: Optional[torch.Tensor] = None,
+                             lse_part: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None,
+                             stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode over the tokens page_table / seq_lens cover, as one split's fp32 partial
+    result: (o_part fp32 [B][Hq][D] normalised, lse_part fp32 [B][Hq]), the inputs
+    lse_combine merges."""
+    _need(q, "q", torch.bfloat16)
+    B, Hq, D = q.shape
+    _need(k_pages, "k_pages", _KV_DTYPES)
+    _need(v_pages, "v_pages", k_pages.dtype, k_pages.shape)
+    num_pages, Hk, P, D2 = k_pages.shape
+    if D2 != D:
+        raise ValueError("head_dim of q and the KV pools differ")
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B][pt_stride]")
+    kv_dtype = _kv_code(k_pages)
+    if kv_dtype == GQA_KV_FP8_E4M3:
+        if k_scale is None or v_scale is None:
+            raise ValueError("fp8 KV needs k_scale and v_scale")
+        _need(k_scale, "k_scale", torch.float32, (num_pages, Hk))
+        _need(v_scale, "v_scale", torch.float32, (num_pages, Hk))
+    pt_stride = page_table.shape[1]
+    if o_part is None:
+        o_part = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    _need(o_part, "o_part", torch.float32, (B, Hq, D))
+    if lse_part is None:
+        lse_part = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    _need(lse_part, "lse_part", torch.float32, (B, Hq))
+    need = gqa_paged_decode_workspace_size(B, Hq, Hk, D, P, pt_stride * P, kv_dtype, num_splits)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = load().gqa_paged_decode_partial(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale), kv_dtype,
+        _ptr(page_table), pt_stride, _ptr(seq_lens), B, Hq, Hk, D, P, num_pages, float(scale),
+        int(num_splits), int(bool(pack_gqa)), _ptr(o_part), _ptr(lse_part), _ptr(workspace),
+        workspace.numel(), _stream(stream))
+    _check("gqa_paged_decode_partial", st)
+    return o_part, lse_part
 
 
 def gqa_paged_decode_static_scratch(q: torch.Tensor, k_pages: torch.Tensor,

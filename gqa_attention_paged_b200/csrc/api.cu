@@ -112,6 +112,96 @@ int sm_count() {
 
 }  // namespace
 
+namespace gqa {
+
+int decode_check_args(const void *q, const void *k_pages, const void *v_pages,
+                      const float *k_scale, const float *v_scale, int kv_dtype,
+                      const int32_t *page_table, int pt_stride, const int32_t *seq_lens, int B,
+                      int Hq, int Hk, int head_dim, int page_size, int num_pages, int num_splits,
+                      const void *out, const float *lse) {
+    if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out) return GQA_ERR_NULL;
+    if (kv_dtype != GQA_KV_BF16 && kv_dtype != GQA_KV_FP8_E4M3) return GQA_ERR_DTYPE;
+    if (kv_dtype == GQA_KV_FP8_E4M3 && (!k_scale || !v_scale || head_dim != 128))
+        return GQA_ERR_DTYPE;
+    if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || Hk > 65535 ||
+        (head_dim != 64 && head_dim != 128) || !valid_page_size(page_size) || num_pages <= 0 ||
+        pt_stride <= 0 || (int64_t)num_pages * Hk * page_size > INT32_MAX ||
+        (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+        !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+        return GQA_ERR_ALIGN;
+    return GQA_OK;
+}
+
+// gqa_paged_decode() and gqa_paged_decode_partial(): out is bf16, or fp32 when out_f32.
+int decode_call(const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
+                const float *v_scale, int kv_dtype, const int32_t *page_table, int pt_stride,
+                const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim, int page_size,
+                int num_pages, float scale, int num_splits, int pack_gqa, void *out, int out_f32,
+                float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    const int chk = decode_check_args(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table,
+                                      pt_stride, seq_lens, B, Hq, Hk, head_dim, page_size,
+                                      num_pages, num_splits, out, lse);
+    if (chk != GQA_OK) return chk;
+    if (!workspace) return GQA_ERR_NULL;
+    const bool sk = use_stream_k(num_splits, B);
+    const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
+    const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                        pt_stride * page_size, kv_dtype,
+                                                        sk ? 0 : S);
+    if (!aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
+    if (B == 0) return GQA_OK;
+
+    const int64_t rows = (int64_t)num_pages * Hk * page_size;
+    CUtensorMap kmap, vmap;
+    const int box_rows = decode_tile_tokens(kv_dtype, page_size);
+    if (encode_kv_map(&kmap, k_pages, kv_dtype, head_dim, rows, box_rows) != GQA_OK ||
+        encode_kv_map(&vmap, v_pages, kv_dtype, head_dim, rows, box_rows) != GQA_OK)
+        return GQA_ERR_LAUNCH;
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    DecodeArgs a;
+    a.q = q;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.page_table = page_table;
+    a.pt_stride = pt_stride;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hk = Hk;
+    a.D = head_dim;
+    a.P = page_size;
+    a.num_pages = num_pages;
+    a.kv_dtype = kv_dtype;
+    a.scale = scale;
+    a.num_splits = S;
+    a.pack_gqa = pack_gqa ? 1 : 0;
+    a.out = out;
+    a.out_f32 = out_f32;
+    a.lse = lse;
+    a.err = reinterpret_cast<int *>(ws);
+    const size_t rows_q = (size_t)B * Hq;
+    a.o_part = S > 1 ? reinterpret_cast<float *>(ws + kWorkspaceHeader) : nullptr;
+    a.lse_part = S > 1 ? reinterpret_cast<float *>(
+                             ws + kWorkspaceHeader +
+                             align_up((size_t)S * rows_q * head_dim * sizeof(float), 256))
+                       : nullptr;
+    a.stream_k = sk ? 1 : 0;
+    a.counters = sk ? reinterpret_cast<int *>(ws + kWorkspaceHeader) : nullptr;
+    a.pieces = sk ? reinterpret_cast<float *>(ws + decode_zero_prefix_bytes(B, Hq)) : nullptr;
+    a.grid = decode_grid();
+    if (launch_decode(a, kmap, vmap, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (S > 1 && launch_lse_combine(a.o_part, a.lse_part, S, (int)rows_q, head_dim, out, lse,
+                                    stream, out_f32) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    return GQA_OK;
+}
+
+}  // namespace gqa
+
 extern "C" {
 
 const char *gqa_status_string(int s) {
@@ -185,71 +275,22 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                      int Hq, int Hk, int head_dim, int page_size, int num_pages, float scale,
                      int num_splits, int pack_gqa, void *out, float *lse, void *workspace,
                      size_t workspace_bytes, cudaStream_t stream) {
-    if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !workspace)
-        return GQA_ERR_NULL;
-    if (kv_dtype != GQA_KV_BF16 && kv_dtype != GQA_KV_FP8_E4M3) return GQA_ERR_DTYPE;
-    if (kv_dtype == GQA_KV_FP8_E4M3 && (!k_scale || !v_scale || head_dim != 128))
-        return GQA_ERR_DTYPE;
-    if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || Hk > 65535 ||
-        (head_dim != 64 && head_dim != 128) || !valid_page_size(page_size) || num_pages <= 0 ||
-        pt_stride <= 0 || (int64_t)num_pages * Hk * page_size > INT32_MAX ||
-        (int64_t)pt_stride * page_size > INT32_MAX)
-        return GQA_ERR_SHAPE;
-    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
-    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
-        !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
-        return GQA_ERR_ALIGN;
-    const bool sk = use_stream_k(num_splits, B);
-    const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
-    const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
-                                                        pt_stride * page_size, kv_dtype,
-                                                        sk ? 0 : S);
-    if (!aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
-    if (B == 0) return GQA_OK;
+    return decode_call(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table, pt_stride,
+                       seq_lens, B, Hq, Hk, head_dim, page_size, num_pages, scale, num_splits,
+                       pack_gqa, out, 0, lse, workspace, workspace_bytes, stream);
+}
 
-    const int64_t rows = (int64_t)num_pages * Hk * page_size;
-    CUtensorMap kmap, vmap;
-    const int box_rows = decode_tile_tokens(kv_dtype, page_size);
-    if (encode_kv_map(&kmap, k_pages, kv_dtype, head_dim, rows, box_rows) != GQA_OK ||
-        encode_kv_map(&vmap, v_pages, kv_dtype, head_dim, rows, box_rows) != GQA_OK)
-        return GQA_ERR_LAUNCH;
-
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    DecodeArgs a;
-    a.q = q;
-    a.k_scale = k_scale;
-    a.v_scale = v_scale;
-    a.page_table = page_table;
-    a.pt_stride = pt_stride;
-    a.seq_lens = seq_lens;
-    a.B = B;
-    a.Hq = Hq;
-    a.Hk = Hk;
-    a.D = head_dim;
-    a.P = page_size;
-    a.num_pages = num_pages;
-    a.kv_dtype = kv_dtype;
-    a.scale = scale;
-    a.num_splits = S;
-    a.pack_gqa = pack_gqa ? 1 : 0;
-    a.out = out;
-    a.lse = lse;
-    a.err = reinterpret_cast<int *>(ws);
-    const size_t rows_q = (size_t)B * Hq;
-    a.o_part = S > 1 ? reinterpret_cast<float *>(ws + kWorkspaceHeader) : nullptr;
-    a.lse_part = S > 1 ? reinterpret_cast<float *>(
-                             ws + kWorkspaceHeader +
-                             align_up((size_t)S * rows_q * head_dim * sizeof(float), 256))
-                       : nullptr;
-    a.stream_k = sk ? 1 : 0;
-    a.counters = sk ? reinterpret_cast<int *>(ws + kWorkspaceHeader) : nullptr;
-    a.pieces = sk ? reinterpret_cast<float *>(ws + decode_zero_prefix_bytes(B, Hq)) : nullptr;
-    a.grid = decode_grid();
-    if (launch_decode(a, kmap, vmap, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
-    if (S > 1 && launch_lse_combine(a.o_part, a.lse_part, S, (int)rows_q, head_dim, out, lse,
-                                    stream) != cudaSuccess)
-        return GQA_ERR_LAUNCH;
-    return GQA_OK;
+int gqa_paged_decode_partial(const void *q, const void *k_pages, const void *v_pages,
+                             const float *k_scale, const float *v_scale, int kv_dtype,
+                             const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                             int B, int Hq, int Hk, int head_dim, int page_size, int num_pages,
+                             float scale, int num_splits, int pack_gqa, float *o_part,
+                             float *lse_part, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+    if (!lse_part) return GQA_ERR_NULL;
+    return decode_call(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table, pt_stride,
+                       seq_lens, B, Hq, Hk, head_dim, page_size, num_pages, scale, num_splits,
+                       pack_gqa, o_part, 1, lse_part, workspace, workspace_bytes, stream);
 }
 
 int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,

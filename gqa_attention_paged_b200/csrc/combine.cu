@@ -10,11 +10,11 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D>
+template <int D, typename OutT>
 __global__ void __launch_bounds__(256) lse_combine_kernel(const float *__restrict__ o_part,
                                                           const float *__restrict__ lse_part,
                                                           int num_splits, int rows,
-                                                          __nv_bfloat16 *__restrict__ out,
+                                                          OutT *__restrict__ out,
                                                           float *__restrict__ lse) {
     constexpr int V = D / 32;
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -48,25 +48,40 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float *__restric
         }
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
-    __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(out + (size_t)row * D + lane * V);
+    if constexpr (sizeof(OutT) == 4) {
+        float2 *dst = reinterpret_cast<float2 *>(out + (size_t)row * D + lane * V);
 #pragma unroll
-    for (int v = 0; v < V; v += 2) dst[v / 2] = __floats2bfloat162_rn(acc[v] * inv, acc[v + 1] * inv);
+        for (int v = 0; v < V; v += 2) dst[v / 2] = make_float2(acc[v] * inv, acc[v + 1] * inv);
+    } else {
+        __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(out + (size_t)row * D + lane * V);
+#pragma unroll
+        for (int v = 0; v < V; v += 2) dst[v / 2] = __floats2bfloat162_rn(acc[v] * inv, acc[v + 1] * inv);
+    }
     if (lane == 0 && lse) lse[row] = W > 0.f ? M + logf(W) : -INFINITY;
 }
 
 }  // namespace
 
 cudaError_t launch_lse_combine(const float *o_part, const float *lse_part, int num_splits,
-                               int rows, int D, void *out, float *lse, cudaStream_t stream) {
+                               int rows, int D, void *out, float *lse, cudaStream_t stream,
+                               int out_f32) {
     if (rows <= 0) return cudaSuccess;
     const int threads = 256;
     const int blocks = (int)(((size_t)rows * 32 + threads - 1) / threads);
-    if (D == 128)
-        lse_combine_kernel<128><<<blocks, threads, 0, stream>>>(
+    if (out_f32) {
+        if (D == 128)
+            lse_combine_kernel<128, float><<<blocks, threads, 0, stream>>>(
+                o_part, lse_part, num_splits, rows, static_cast<float *>(out), lse);
+        else
+            lse_combine_kernel<64, float><<<blocks, threads, 0, stream>>>(
+                o_part, lse_part, num_splits, rows, static_cast<float *>(out), lse);
+    } else if (D == 128) {
+        lse_combine_kernel<128, __nv_bfloat16><<<blocks, threads, 0, stream>>>(
             o_part, lse_part, num_splits, rows, static_cast<__nv_bfloat16 *>(out), lse);
-    else
-        lse_combine_kernel<64><<<blocks, threads, 0, stream>>>(
+    } else {
+        lse_combine_kernel<64, __nv_bfloat16><<<blocks, threads, 0, stream>>>(
             o_part, lse_part, num_splits, rows, static_cast<__nv_bfloat16 *>(out), lse);
+    }
     return cudaGetLastError();
 }
 

@@ -102,6 +102,17 @@ __device__ __forceinline__ int clamp_len(int L, int Lmax, int *err) {
     return L;
 }
 
+// Output stores: bf16 (the decode's result) or fp32 (the normalised partial of
+// gqa_paged_decode_partial, an input of lse_combine).  idx counts elements.
+__device__ __forceinline__ void store_out1(void *out, int f32, size_t idx, float v) {
+    if (f32) reinterpret_cast<float *>(out)[idx] = v;
+    else reinterpret_cast<__nv_bfloat16 *>(out)[idx] = __float2bfloat16(v);
+}
+__device__ __forceinline__ void store_out2(void *out, int f32, size_t idx, float v0, float v1) {
+    if (f32) reinterpret_cast<float2 *>(out)[idx / 2] = make_float2(v0, v1);
+    else reinterpret_cast<__nv_bfloat162 *>(out)[idx / 2] = __floats2bfloat162_rn(v0, v1);
+}
+
 // One consumer warp's attention state for up to 8*NT packed heads of one kv head:
 // q fragments, the running max / sum per head, and O^T accumulators.
 //   fragment lane (gq = lane / 4, cq = lane % 4) holds heads 8*nt + 2*cq (+1) and, for
@@ -606,8 +617,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         const float lse_v = Ls > 0.f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
         const size_t row = (size_t)b * a.Hq + head_lo + h;
         if (a.num_splits == 1) {
-            reinterpret_cast<__nv_bfloat162 *>(a.out)[(row * D + d) / 2] =
-                __floats2bfloat162_rn(o0 * inv, o1 * inv);
+            store_out2(a.out, a.out_f32, row * D + d, o0 * inv, o1 * inv);
             if (d == 0 && a.lse) a.lse[row] = lse_v;
         } else {
             const size_t prow = (size_t)split * rows_total + row;
@@ -693,8 +703,8 @@ __device__ __forceinline__ void flat_next(FlatPos &p, const int *pre, int U) {
 // other.
 template <int D, int HW>
 __device__ __forceinline__ void merge_pieces(const float *pieces, long long wfirst, long long wlast,
-                                          int slot_floats, int hpc, int nh, __nv_bfloat16 *out_rows,
-                                          float *lse_rows, int lane) {
+                                          int slot_floats, int hpc, int nh, void *out, int out_f32,
+                                          size_t out0, float *lse_rows, int lane) {
     constexpr int DV = D / 32;
     float Mh[HW], Wh[HW], acc[HW][DV];
 #pragma unroll
@@ -735,9 +745,9 @@ __device__ __forceinline__ void merge_pieces(const float *pieces, long long wfir
     for (int h = 0; h < HW; ++h) {
         if (h >= nh) continue;
         const float inv = 1.f / Wh[h];
-        __nv_bfloat162 *dst = reinterpret_cast<__nv_bfloat162 *>(out_rows + (size_t)h * D + DV * lane);
+        const size_t e0 = out0 + (size_t)h * D + DV * lane;
 #pragma unroll
-        for (int v = 0; v < DV; v += 2) dst[v / 2] = __floats2bfloat162_rn(acc[h][v] * inv, acc[h][v + 1] * inv);
+        for (int v = 0; v < DV; v += 2) store_out2(out, out_f32, e0 + v, acc[h][v] * inv, acc[h][v + 1] * inv);
         if (lane == 0 && lse_rows) lse_rows[h] = Mh[h] + logf(Wh[h]);
     }
 }
@@ -826,8 +836,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     // Sequences with no tokens have no tiles: their outputs are written here (zeros, -inf).
     for (int b = blockIdx.x; b < B; b += gridDim.x) {
         if (pre[b + 1] != pre[b]) continue;
-        __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(a.out) + (size_t)b * a.Hq * D;
-        for (int e = threadIdx.x; e < a.Hq * D; e += kThreads) ob[e] = __float2bfloat16(0.f);
+        for (int e = threadIdx.x; e < a.Hq * D; e += kThreads)
+            store_out1(a.out, a.out_f32, (size_t)b * a.Hq * D + e, 0.f);
         if (a.lse)
             for (int e = threadIdx.x; e < a.Hq; e += kThreads) a.lse[(size_t)b * a.Hq + e] = -INFINITY;
     }
@@ -979,11 +989,11 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
                     const int h = nt * 8 + 2 * cq + jj;
                     if (h >= nh) continue;
                     const float inv = st.l[nt][jj] > 0.f ? 1.f / st.l[nt][jj] : 0.f;
-                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) + (row0 + h) * D;
+                    const size_t e0 = (row0 + h) * D;
 #pragma unroll
                     for (int dt = 0; dt < KT; ++dt) {
-                        dst[WA::dim0(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj] * inv);
-                        dst[WA::dim1(dt, gq)] = __float2bfloat16(st.o[nt][dt][jj + 2] * inv);
+                        store_out1(a.out, a.out_f32, e0 + WA::dim0(dt, gq), st.o[nt][dt][jj] * inv);
+                        store_out1(a.out, a.out_f32, e0 + WA::dim1(dt, gq), st.o[nt][dt][jj + 2] * inv);
                     }
                     if (gq == 0 && a.lse)
                         a.lse[row0 + h] = st.l[nt][jj] > 0.f
@@ -1025,8 +1035,8 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
                 if (last) {
                     __threadfence();
                     merge_pieces<D, HW>(a.pieces, wfirst, wlast, slot_floats, heads_per_cta, nh,
-                                        reinterpret_cast<__nv_bfloat16 *>(a.out) + row0 * D,
-                                        a.lse ? a.lse + row0 : nullptr, lane);
+                                        a.out, a.out_f32, row0 * D, a.lse ? a.lse + row0 : nullptr,
+                                        lane);
                     if (lane == 0) *ctr = 0;  // ready for the next launch
                 }
             }
@@ -1115,8 +1125,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < kMergeWarps; ++w) sum += part[w][d];
-            reinterpret_cast<__nv_bfloat16 *>(a.out)[((size_t)b * a.Hq + head_lo + h) * D + d] =
-                __float2bfloat16(sum * inv);
+            store_out1(a.out, a.out_f32, ((size_t)b * a.Hq + head_lo + h) * D + d, sum * inv);
         }
         if (threadIdx.x == 0 && a.lse) a.lse[(size_t)b * a.Hq + head_lo + h] = M + logf(W);
         __syncthreads();  // part[] and lse_s[] are reused by the next unit

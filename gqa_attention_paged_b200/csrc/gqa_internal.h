@@ -22,7 +22,8 @@ struct DecodeArgs {
     float scale;
     int num_splits;
     int pack_gqa;
-    void *out;
+    void *out;        // bf16 [B][Hq][D], or fp32 when out_f32
+    int out_f32;      // 1: write the normalised result in fp32 (gqa_paged_decode_partial)
     float *lse;
     float *o_part, *lse_part;  // scratch for num_splits > 1
     int *err;
@@ -66,14 +67,24 @@ inline size_t decode_zero_prefix_bytes(int B, int Hq) {
     return kWorkspaceHeader + ((size_t)B * Hq * sizeof(int) + 255) / 256 * 256;
 }
 
+// Host-side checks of gqa_paged_decode()'s arguments other than the workspace: GQA_OK or
+// the status the call returns (nothing is enqueued by a call that fails them).
+int decode_check_args(const void *q, const void *k_pages, const void *v_pages,
+                      const float *k_scale, const float *v_scale, int kv_dtype,
+                      const int32_t *page_table, int pt_stride, const int32_t *seq_lens, int B,
+                      int Hq, int Hk, int head_dim, int page_size, int num_pages, int num_splits,
+                      const void *out, const float *lse);
+
 // Launch the decode kernel on `stream` (for launches whose units are cut into many pieces,
 // followed by the kernel that merges the pieces).  The tensor maps describe the
 // K and V pools as 2-D arrays [num_pages*Hk*P rows][D].
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);
 
+// out is bf16 [rows][D], or fp32 when out_f32.
 cudaError_t launch_lse_combine(const float *o_part, const float *lse_part, int num_splits,
-                               int rows, int D, void *out, float *lse, cudaStream_t stream);
+                               int rows, int D, void *out, float *lse, cudaStream_t stream,
+                               int out_f32 = 0);
 
 cudaError_t launch_gather(const void *k_pages, const void *v_pages, const int32_t *page_table,
                           int pt_stride, const int32_t *seq_lens, const int64_t *cu_kv, int B,

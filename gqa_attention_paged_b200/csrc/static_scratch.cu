@@ -46,24 +46,25 @@ extern "C" int gqa_paged_decode_static_scratch(
     const float *v_scale, int kv_dtype, const int32_t *page_table, int pt_stride,
     const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim, int page_size, int num_pages,
     float scale, int num_splits, int pack_gqa, void *out, float *lse, cudaStream_t stream) {
-    // Size check first (only for arguments gqa_paged_decode would accept; it reports the
-    // rest itself): the scratch this call needs must fit the fixed array.
-    if (B > 0 && Hq > 0 && Hk > 0 && head_dim > 0 && page_size > 0 && pt_stride > 0 &&
-        num_splits >= 0 && num_splits <= GQA_MAX_SPLITS &&
-        (int64_t)pt_stride * page_size <= INT32_MAX) {
-        const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
-                                                            pt_stride * page_size, kv_dtype,
-                                                            num_splits);
-        if (need > (size_t)GQA_STATIC_SCRATCH_BYTES) return GQA_ERR_WORKSPACE;
-    }
+    // gqa_paged_decode()'s own argument checks first, so a call it would reject queues
+    // nothing (not even the memset below); then the size check: the scratch this call
+    // needs must fit the fixed array.
+    const int chk = gqa::decode_check_args(q, k_pages, v_pages, k_scale, v_scale, kv_dtype,
+                                           page_table, pt_stride, seq_lens, B, Hq, Hk, head_dim,
+                                           page_size, num_pages, num_splits, out, lse);
+    if (chk != GQA_OK) return chk;
+    const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                        pt_stride * page_size, kv_dtype,
+                                                        num_splits);
+    if (need > (size_t)GQA_STATIC_SCRATCH_BYTES) return GQA_ERR_WORKSPACE;
+    if (B == 0) return GQA_OK;
     void *ws = nullptr;
     const int st = scratch_address(&ws);
     if (st != GQA_OK) return st;
     // The array keeps the previous call's contents.  What must start at zero is cleared:
     // the error word and the balanced schedule's merge counters (split partials and merge
     // pieces are fully rewritten by every call that reads them).
-    size_t zero = sizeof(int);
-    if (B > 0 && Hq > 0) zero = gqa::decode_zero_prefix_bytes(B, Hq);
+    size_t zero = gqa::decode_zero_prefix_bytes(B, Hq);
     if (zero > (size_t)GQA_STATIC_SCRATCH_BYTES) zero = (size_t)GQA_STATIC_SCRATCH_BYTES;
     if (cudaMemsetAsync(ws, 0, zero, stream) != cudaSuccess) return GQA_ERR_LAUNCH;
     return gqa_paged_decode(q, k_pages, v_pages, k_scale, v_scale, kv_dtype, page_table,

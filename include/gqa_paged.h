@@ -149,6 +149,36 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
                      size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Decode over this rank's share of each sequence's history, for a sequence whose pages are
+ * spread over several GPUs: every GPU computes the attention of the new query token over
+ * the tokens it holds, the GPUs exchange these partial results, and each merges them with
+ * lse_combine() ("FasterTransformer source tour", section 6.1: splitting a context too
+ * long for one device across devices; the merge is the NumSplits log-sum-exp merge of
+ * "解锁GQA性能潜力：从批量大小敏感性到高效优化实践", section
+ * "核心参数调优：PackGQA与NumSplits的协同舞蹈").
+ *
+ * Arguments and checks are gqa_paged_decode()'s: page_table / seq_lens describe the
+ * tokens THIS call covers (its rows of the page table and the number of those tokens per
+ * sequence, 0 for a sequence with none here).  The results are written in fp32 instead of
+ * bf16, in the form lse_combine() takes for one split:
+ *   o_part    fp32 [B][Hq][head_dim]: softmax-normalised attention over the covered tokens
+ *             (0 for a sequence with none), 16-byte aligned
+ *   lse_part  fp32 [B][Hq]: natural-log log-sum-exp of the covered scores (-inf for a
+ *             sequence with none); required (NULL gives GQA_ERR_NULL)
+ * Stacking the o_part / lse_part of R such calls (R ranks, or R disjoint page ranges) as
+ * [R][B*Hq][head_dim] / [R][B*Hq] and passing them to lse_combine(num_splits = R) gives
+ * the decode over all their tokens.  Workspace: gqa_paged_decode_workspace_size() with
+ * the same arguments.
+ */
+int gqa_paged_decode_partial(const void *q, const void *k_pages, const void *v_pages,
+                             const float *k_scale, const float *v_scale, int kv_dtype,
+                             const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                             int B, int Hq, int Hk, int head_dim, int page_size, int num_pages,
+                             float scale, int num_splits, int pack_gqa, float *o_part,
+                             float *lse_part, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/*
  * Largest scratch gqa_paged_decode_static_scratch() can use: its fixed array's size.
  */
 #define GQA_STATIC_SCRATCH_BYTES (16u << 20)
@@ -177,13 +207,18 @@ int gqa_paged_decode(const void *q, const void *k_pages, const void *v_pages,
  *   - Device-side errors (out-of-range page entries, a bounded wait that ran out) are
  *     recorded in the array's error word but cannot be read back through this entry
  *     point.  Use gqa_paged_decode() with a workspace when those reports are needed.
+ *   - The cached address belongs to the device's context as it was at the first call:
+ *     calls after cudaDeviceReset() on that device are not supported.
  *
  * Arguments are gqa_paged_decode()'s, minus workspace / workspace_bytes.  Returns what
- * gqa_paged_decode() returns.  Also returns GQA_ERR_WORKSPACE, with nothing enqueued,
- * when the call needs more than GQA_STATIC_SCRATCH_BYTES of scratch, i.e. when
+ * gqa_paged_decode() returns; its argument checks run first, so a call it rejects
+ * enqueues nothing.  Also returns GQA_ERR_WORKSPACE, with nothing enqueued, when the call
+ * needs more than GQA_STATIC_SCRATCH_BYTES of scratch, i.e. when
  * gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
  * pt_stride * page_size, kv_dtype, num_splits) exceeds it.  Lower num_splits or the
- * batch to fit.
+ * batch to fit.  One case never fits with num_splits = 0: groups of more than 8 query
+ * heads per kv head at head_dim 128 (the balanced schedule's merge pieces alone take
+ * about 21 MB); pass num_splits >= 1 for those.
  */
 int gqa_paged_decode_static_scratch(const void *q, const void *k_pages, const void *v_pages,
                                     const float *k_scale, const float *v_scale, int kv_dtype,

@@ -151,3 +151,32 @@ def test_prefill_rejects_bad_arguments_on_the_host():
     assert call(Hq=6, Hk=4) == -2
     assert call(wsb=16) == -5
     assert call(q=_fake(0x10008)) == -9
+
+
+def _static(**kw):
+    args = dict(q=_fake(), k=_fake(), v=_fake(), ks=None, vs=None, kvd=0, pt=_fake(), pts=128,
+                sl=_fake(), B=16, Hq=32, Hk=8, D=128, P=16, npg=4096, scale=0.088, S=0, pack=1,
+                out=_fake(), lse=None, st=None)
+    args.update(kw)
+    return binding.load().gqa_paged_decode_static_scratch(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    # gqa_paged_decode's own checks come first: nothing (not even the scratch memset) is
+    # queued for a call it rejects
+    (dict(q=None), -1), (dict(kvd=7), -3), (dict(Hq=30), -2), (dict(S=65), -4),
+    (dict(out=_fake(0x10008)), -9),
+    # then the size check: 64 splits of B=64 need more than the fixed array
+    (dict(B=64, S=64), -5),
+    # groups of more than 8 heads at head_dim 128 never fit the balanced schedule's pieces
+    (dict(Hq=128, Hk=8, S=0), -5), (dict(Hq=16, Hk=1, S=0), -5),
+])
+def test_static_scratch_rejects_on_the_host(kw, status):
+    """These pointers are never dereferenced: every rejection happens on the host."""
+    assert _static(**kw) == status
+
+
+def test_static_scratch_fits_groups_above_8_with_splits():
+    lib = binding.load()
+    assert lib.gqa_paged_decode_workspace_size(16, 128, 8, 128, 16, 2048, 0, 0) > 16 << 20
+    assert lib.gqa_paged_decode_workspace_size(16, 128, 8, 128, 16, 2048, 0, 2) <= 16 << 20

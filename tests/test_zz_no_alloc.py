@@ -1,10 +1,15 @@
 """gqa_paged_decode_static_scratch: decode for callers that cannot allocate device memory
 (an engine plugin's enqueue, an allocation-free real-time loop, a host whose device memory
-belongs to another allocator).  It keeps its split partials in a fixed array inside the
-library instead of a caller workspace.  Checked here through the C ABI against
-gqa_paged_decode on the same inputs, within the bf16 tolerance of the other tests
-(|err| <= 2e-3 + 1e-2 |ref|), on two calls in a row with different shapes, so the second
-call runs on the array as the first one left it.
+belongs to another allocator).  It keeps its split partials, merge pieces and merge
+counters in a fixed array inside the library instead of a caller workspace.
+
+Checked here through the C ABI against gqa_paged_decode (fresh workspace) and against the
+fp64 oracle, within the bf16 tolerance of the other tests (|err| <= 2e-3 + 1e-2 |ref|),
+on calls in a row on the one shared array: every call runs on the array as the previous
+call left it.  The sequence covers the split schedule, then the balanced schedule (whose
+merge counters sit where the previous call's split partials were), the balanced schedule
+with its separate piece merge (a few long sequences), and a repeat of the first balanced
+call, which must give the same bits.
 
 This file is named to be collected last."""
 import ctypes
@@ -14,7 +19,7 @@ import pytest
 import torch
 
 from gqa_attention_paged_b200 import binding, inputs
-from tests._util import bf16_tol_ok, err_report
+from tests._util import bf16_tol_ok, err_report, oracle_decode
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -48,21 +53,50 @@ def _dev(case):
     return d
 
 
+def _check(case, d, S, tag):
+    """One static-scratch call, compared with the workspace call and with the oracle."""
+    ref_o, ref_l = binding.gqa_paged_decode(d["q"], d["k"], d["v"], d["pt"], d["sl"],
+                                            case.scale, num_splits=S,
+                                            k_scale=d.get("ks"), v_scale=d.get("vs"))
+    st, out, lse = _static_call(d, case, S)
+    assert st == 0, f"{tag}: {binding.status_string(st)}"
+    o = out.float().cpu().numpy()
+    ro = ref_o.float().cpu().numpy()
+    ok, bad = bf16_tol_ok(o, ro)
+    assert ok, f"{tag} vs workspace call: {err_report(o, ro)} bad={int(bad.sum())}"
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_l.cpu().numpy(), rtol=1e-4, atol=2e-3,
+                               err_msg=f"{tag} lse vs workspace call")
+    oo, ol = oracle_decode(case)
+    ok, bad = bf16_tol_ok(o, oo)
+    assert ok, f"{tag} vs oracle: {err_report(o, oo)} bad={int(bad.sum())}"
+    np.testing.assert_allclose(lse.cpu().numpy(), ol, rtol=1e-4, atol=2e-3,
+                               err_msg=f"{tag} lse vs oracle")
+    return out, lse
+
+
 def test_static_scratch_matches_workspace_decode_two_calls_in_a_row():
     calls = [(inputs.llama7b_decode(seed=11), 4),              # 4 splits of a ragged batch
              (inputs.make_decode_case(3, 16, 2, 64, 32, [300, 7, 129], seed=12), 3)]
     for i, (case, S) in enumerate(calls):
-        d = _dev(case)
-        ref_o, ref_l = binding.gqa_paged_decode(d["q"], d["k"], d["v"], d["pt"], d["sl"],
-                                                case.scale, num_splits=S,
-                                                k_scale=d.get("ks"), v_scale=d.get("vs"))
-        st, out, lse = _static_call(d, case, S)
-        assert st == 0, binding.status_string(st)
-        ro, o = ref_o.float().cpu().numpy(), out.float().cpu().numpy()
-        ok, bad = bf16_tol_ok(o, ro)
-        assert ok, f"call {i}: {err_report(o, ro)} bad={int(bad.sum())}"
-        rl, l = ref_l.cpu().numpy(), lse.cpu().numpy()
-        np.testing.assert_allclose(l, rl, rtol=1e-4, atol=2e-3, err_msg=f"call {i}")
+        _check(case, _dev(case), S, f"call {i}")
+
+
+def test_static_scratch_balanced_after_split_calls():
+    """split (S=4) -> balanced -> balanced with the separate piece merge -> balanced again.
+    The first balanced call's merge counters occupy bytes the split call's partials
+    overwrote, so they must be cleared by the call itself."""
+    ragged = inputs.llama7b_decode(seed=21)
+    few_long = inputs.make_decode_case(2, 32, 8, 128, 16, [4096, 3001], seed=22)
+    d_r, d_f = _dev(ragged), _dev(few_long)
+    # the second balanced shape really takes the separate piece merge
+    assert binding.gqa_paged_decode_kernel_launches(2, 32, 8, 128, 16, 4096, 0, 0) == 2
+    assert binding.gqa_paged_decode_kernel_launches(16, 32, 8, 128, 16, 2048, 0, 0) == 1
+    _check(ragged, d_r, 4, "split S=4")
+    o1, l1 = _check(ragged, d_r, 0, "balanced after split")
+    _check(few_long, d_f, 0, "balanced, separate piece merge")
+    o2, l2 = _check(ragged, d_r, 0, "balanced again")
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)), "repeated balanced calls differ"
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))
 
 
 def test_static_scratch_rejects_calls_that_do_not_fit():
