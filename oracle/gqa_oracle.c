@@ -435,3 +435,184 @@ void oracle_append_kv(void *k_pages, void *v_pages, float *k_scale, float *v_sca
         }
     }
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Page-level top-K sparse decode: the decode stage of RocketKV as the page
+ * "TensorRT-LLM 如何用 sparse_attention_config 配置 Sparse Attention 降低长上下文推理开销"
+ * (RocketKV configuration section) describes it: an auxiliary KT cache scores the pages,
+ * and the decode attends to the `topk` best pages plus the most recent `window` tokens
+ * only.  Readings taken where the page is silent:
+ *   - KT entry of (page, kv head): the element-wise minimum and maximum of the page's key
+ *     vectors over its valid tokens.  kt[page][kvh][d][0] = min, [1] = max.
+ *   - Score of a page for query head h: sum over d of max(q_d * min_d, q_d * max_d), the
+ *     largest q.k over the box [min, max] and so an upper bound of q.k for every key of
+ *     the page.  Score for a kv head: the sum of its g query heads' scores.  Computed in
+ *     fp32, the decision's precision on the GPU: per head with d ascending, then heads
+ *     ascending.  Every product of two bf16 values is exact in fp32, so both sides round
+ *     the same sums the same way.
+ *   - The selection unit is one KV-cache page (the page's sparse page_size taken equal to
+ *     the cache's page size; the page asks for a power of two, which 16/32/64 are), and the
+ *     query channels used are all head_dim of them (the page advises topr = head_dim).
+ *   - Window: the pages holding any of the last `window` tokens are always attended.
+ *     Among the earlier pages the `topk` highest scores are chosen, equal scores going to
+ *     the lower logical page; with no more than `topk` earlier pages, all are chosen.
+ *   - The attention itself is plain softmax attention over the tokens of the chosen
+ *     pages (attend_row above), in logical page order.
+ * ------------------------------------------------------------------------------------- */
+
+/* KT entries of every page sequence b references: for page p < ceil(L/P), over its
+ * n = min(P, L - p*P) valid tokens.  kt: double [num_pages][Hk][D][2] (caller-owned;
+ * entries of unreferenced pages are left as they are). */
+void oracle_kt_build(const uint16_t *k_pages, const int32_t *page_table, int pt_stride,
+                     const int32_t *seq_lens, int B, int Hk, int D, int P, double *kt)
+{
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        int np = (L + P - 1) / P;
+        for (int p = 0; p < np; ++p) {
+            int64_t phys = page_table[(int64_t)b * pt_stride + p];
+            int n = L - p * P < P ? L - p * P : P;
+            for (int kvh = 0; kvh < Hk; ++kvh)
+                for (int d = 0; d < D; ++d) {
+                    double mn = INFINITY, mx = -INFINITY;
+                    for (int t = 0; t < n; ++t) {
+                        double v = kv_value(k_pages, 0, NULL, Hk, P, D, phys, kvh, t, d);
+                        if (v < mn)
+                            mn = v;
+                        if (v > mx)
+                            mx = v;
+                    }
+                    double *e = kt + ((phys * Hk + kvh) * (int64_t)D + d) * 2;
+                    e[0] = mn;
+                    e[1] = mx;
+                }
+        }
+    }
+}
+
+/* Page scores: scores[b][kvh][p] for p < ceil(L_b/P) (fp32, as defined above); entries
+ * at or past ceil(L_b/P) are set to -inf.  kt as built by oracle_kt_build. */
+void oracle_page_scores(const uint16_t *q, const double *kt, const int32_t *page_table,
+                        int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk, int D,
+                        int P, float *scores)
+{
+    int g = Hq / Hk;
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        int np = (L + P - 1) / P;
+        for (int kvh = 0; kvh < Hk; ++kvh)
+            for (int p = 0; p < pt_stride; ++p) {
+                float *dst = scores + ((int64_t)b * Hk + kvh) * pt_stride + p;
+                if (p >= np) {
+                    *dst = -INFINITY;
+                    continue;
+                }
+                int64_t phys = page_table[(int64_t)b * pt_stride + p];
+                const double *e = kt + (phys * Hk + kvh) * (int64_t)D * 2;
+                float total = 0.0f;
+                for (int j = 0; j < g; ++j) {
+                    int h = kvh * g + j;
+                    float sh = 0.0f;
+                    for (int d = 0; d < D; ++d) {
+                        float qd = bf16_bits_to_f32(q[((int64_t)b * Hq + h) * D + d]);
+                        float lo = qd * (float)e[2 * d], hi = qd * (float)e[2 * d + 1];
+                        sh = sh + (lo > hi ? lo : hi);
+                    }
+                    total = total + sh;
+                }
+                *dst = total;
+            }
+    }
+}
+
+/* Selection from the scores: sel[b][kvh][0 .. nsel-1] = the chosen logical pages in
+ * ascending order (window pages included), nsel[b][kvh] their count.  sel has pt_stride
+ * entries per (b, kvh). */
+void oracle_sparse_select(const float *scores, const int32_t *seq_lens, int B, int Hk,
+                          int pt_stride, int P, int topk, int window, int32_t *sel,
+                          int32_t *nsel)
+{
+    char *take = (char *)malloc((size_t)pt_stride + 1);
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        int np = (L + P - 1) / P;
+        int lo = L - window > 0 ? L - window : 0;
+        int wp = window > 0 ? lo / P : np; /* first page holding a window token */
+        if (wp > np)
+            wp = np;
+        for (int kvh = 0; kvh < Hk; ++kvh) {
+            const float *s = scores + ((int64_t)b * Hk + kvh) * pt_stride;
+            for (int p = 0; p < np; ++p)
+                take[p] = p >= wp || wp <= topk;
+            if (wp > topk) {
+                /* topk rounds of "best remaining": highest score, then lowest page */
+                for (int k = 0; k < topk; ++k) {
+                    int best = -1;
+                    for (int p = 0; p < wp; ++p) {
+                        if (take[p])
+                            continue;
+                        if (best < 0 || s[p] > s[best])
+                            best = p;
+                    }
+                    take[best] = 1;
+                }
+            }
+            int32_t *out = sel + ((int64_t)b * Hk + kvh) * pt_stride;
+            int n = 0;
+            for (int p = 0; p < np; ++p)
+                if (take[p])
+                    out[n++] = p;
+            nsel[(int64_t)b * Hk + kvh] = n;
+        }
+    }
+    free(take);
+}
+
+/* Attention of every query head over the tokens of its kv head's chosen pages (sel /
+ * nsel as from oracle_sparse_select), in fp64.  out [B][Hq][D], lse [B][Hq]. */
+void oracle_sparse_decode(const uint16_t *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                          const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                          int B, int Hq, int Hk, int D, int P, double scale, const int32_t *sel,
+                          const int32_t *nsel, double *out, double *lse)
+{
+    int g = Hq / Hk;
+    int max_L = 0;
+    for (int b = 0; b < B; ++b)
+        if (seq_lens[b] > max_L)
+            max_L = seq_lens[b];
+#pragma omp parallel
+    {
+        double *K = (double *)malloc(sizeof(double) * ((size_t)max_L * D + 1));
+        double *V = (double *)malloc(sizeof(double) * ((size_t)max_L * D + 1));
+        double *s = (double *)malloc(sizeof(double) * ((size_t)max_L + 1));
+        double *qd = (double *)malloc(sizeof(double) * (size_t)D);
+#pragma omp for collapse(2) schedule(dynamic)
+        for (int b = 0; b < B; ++b)
+            for (int kvh = 0; kvh < Hk; ++kvh) {
+                int L = seq_lens[b];
+                const int32_t *ps = sel + ((int64_t)b * Hk + kvh) * pt_stride;
+                int n = 0; /* tokens gathered */
+                for (int i = 0; i < nsel[(int64_t)b * Hk + kvh]; ++i) {
+                    int p = ps[i];
+                    int64_t phys = page_table[(int64_t)b * pt_stride + p];
+                    int cnt = L - p * P < P ? L - p * P : P;
+                    for (int t = 0; t < cnt; ++t, ++n)
+                        for (int d = 0; d < D; ++d) {
+                            K[(int64_t)n * D + d] = kv_value(k_pages, 0, NULL, Hk, P, D, phys, kvh, t, d);
+                            V[(int64_t)n * D + d] = kv_value(v_pages, 0, NULL, Hk, P, D, phys, kvh, t, d);
+                        }
+                }
+                for (int j = 0; j < g; ++j) {
+                    int h = kvh * g + j;
+                    for (int d = 0; d < D; ++d)
+                        qd[d] = oracle_bf16_to_f64(q[((int64_t)b * Hq + h) * D + d]);
+                    attend_row(qd, K, V, 0, n, D, scale, s, out + ((int64_t)b * Hq + h) * D,
+                               lse + (int64_t)b * Hq + h);
+                }
+            }
+        free(K);
+        free(V);
+        free(s);
+        free(qd);
+    }
+}

@@ -53,6 +53,19 @@ def lib():
         L.oracle_append_kv.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P,
                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        _P, _P]
+        L.oracle_kt_build.restype = None
+        L.oracle_kt_build.argtypes = [_P, _P, ctypes.c_int, _P, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, _P]
+        L.oracle_page_scores.restype = None
+        L.oracle_page_scores.argtypes = [_P, _P, _P, ctypes.c_int, _P, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, _P]
+        L.oracle_sparse_select.restype = None
+        L.oracle_sparse_select.argtypes = [_P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P]
+        L.oracle_sparse_decode.restype = None
+        L.oracle_sparse_decode.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_double, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -227,3 +240,69 @@ def append_kv(k_pages, v_pages, page_table, seq_lens, k_new, v_new, k_scale=None
                            vs.ctypes.data_as(_P) if fp8 else None, 1 if fp8 else 0, ptp,
                            pt.shape[1], slp, len(sl), Hk, D, P, knp, vnp)
     return kp, vp, ks, vs
+
+
+# ---------------------------------------------------------------------------------------
+# Page-level top-K sparse decode (see the readings in gqa_oracle.c).
+
+def kt_build(k_pages, page_table, seq_lens, kt=None):
+    """KT cache entries (min, max of the keys over each referenced page's valid tokens):
+    returns double [num_pages][Hk][D][2]; entries of unreferenced pages are NaN (or those
+    of `kt` when given)."""
+    num_pages, Hk, P, D = k_pages.shape
+    if k_pages.dtype != np.uint16:
+        raise TypeError("the KT cache is built from bf16 pools")
+    out = np.full((num_pages, Hk, D, 2), np.nan) if kt is None else np.array(kt, np.float64, copy=True)
+    kp, kp_p = _c(k_pages, np.uint16)
+    pt, pt_p = _c(page_table, np.int32)
+    sl, sl_p = _c(seq_lens, np.int32)
+    lib().oracle_kt_build(kp_p, pt_p, pt.shape[1], sl_p, len(sl), Hk, D, P, out.ctypes.data_as(_P))
+    return out
+
+
+def page_scores(q, kt, page_table, seq_lens, page_size):
+    """fp32 page scores [B][Hk][pt_stride] (-inf past each sequence's pages)."""
+    B, Hq, D = q.shape
+    Hk = kt.shape[1]
+    qq, q_p = _c(q, np.uint16)
+    k, k_p = _c(kt, np.float64)
+    pt, pt_p = _c(page_table, np.int32)
+    sl, sl_p = _c(seq_lens, np.int32)
+    out = np.zeros((B, Hk, pt.shape[1]), np.float32)
+    lib().oracle_page_scores(q_p, k_p, pt_p, pt.shape[1], sl_p, B, Hq, Hk, D, page_size,
+                             out.ctypes.data_as(_P))
+    return out
+
+
+def sparse_select(scores, seq_lens, page_size, topk, window):
+    """Chosen logical pages per (sequence, kv head): returns (sel int32 [B][Hk][pt_stride],
+    nsel int32 [B][Hk]); sel[b][j][:nsel[b][j]] ascending."""
+    B, Hk, pts = scores.shape
+    sc, sc_p = _c(scores, np.float32)
+    sl, sl_p = _c(seq_lens, np.int32)
+    sel = np.full((B, Hk, pts), -1, np.int32)
+    nsel = np.zeros((B, Hk), np.int32)
+    lib().oracle_sparse_select(sc_p, sl_p, B, Hk, pts, page_size, int(topk), int(window),
+                               sel.ctypes.data_as(_P), nsel.ctypes.data_as(_P))
+    return sel, nsel
+
+
+def sparse_decode(q, k_pages, v_pages, page_table, seq_lens, scale, sel, nsel):
+    """fp64 attention over the chosen pages: returns (out [B][Hq][D], lse [B][Hq])."""
+    B, Hq, D = q.shape
+    num_pages, Hk, P, _ = k_pages.shape
+    qq, q_p = _c(q, np.uint16)
+    kp, kp_p = _c(k_pages, np.uint16)
+    vp, vp_p = _c(v_pages, np.uint16)
+    pt, pt_p = _c(page_table, np.int32)
+    sl, sl_p = _c(seq_lens, np.int32)
+    se = np.full((B, Hk, pt.shape[1]), -1, np.int32)
+    se[:, :, :sel.shape[2]] = sel[:, :, :pt.shape[1]]
+    se, se_p = _c(se, np.int32)
+    ns, ns_p = _c(nsel, np.int32)
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    lib().oracle_sparse_decode(q_p, kp_p, vp_p, pt_p, pt.shape[1], sl_p, B, Hq, Hk, D, P,
+                               float(scale), se_p, ns_p, out.ctypes.data_as(_P),
+                               lse.ctypes.data_as(_P))
+    return out, lse

@@ -1,8 +1,8 @@
 """Plant plausible mistakes in a COPY of the oracle source and check that a pin catches
 each one.  This shows the pins in test_oracle_pins.py and test_append_cpu.py constrain
 every step of the oracle (head map, page/slot indexing, scale, softmax, lse, split
-boundaries, merge, decoders, causal bound, KV append position, e4m3 encoding and the
-append scale).  The real oracle source is never modified."""
+boundaries, merge, decoders, causal bound, KV append position, e4m3 encoding, the
+append scale, and the sparse decode's KT entries, page scores, selection and gather).  The real oracle source is never modified."""
 import os
 import subprocess
 import tempfile
@@ -14,6 +14,7 @@ from oracle import build as obuild
 from oracle import oracle
 from tests import test_append_cpu as append_pins
 from tests import test_oracle_pins as pins
+from tests import test_sparse_cpu as sparse_pins
 
 MUTANTS = {
     "head_map_interleaved": ("int h = kvh * g + j;\n                    for (int d = 0; d < D; ++d)\n                        qd[d] = oracle_bf16_to_f64(q[((int64_t)b",
@@ -44,13 +45,24 @@ MUTANTS = {
     "append_scale_not_448": ("scale[si] = amax > 0.0f ? amax / 448.0f : 1.0f;",
                              "scale[si] = amax > 0.0f ? amax / 240.0f : 1.0f;"),
     "append_keeps_no_scale": ("if (slot == 0) {\n                    float amax", "if (slot >= 0) {\n                    float amax"),
+    "kt_over_all_slots": ("int n = L - p * P < P ? L - p * P : P;\n            for (int kvh",
+                          "int n = P;\n            for (int kvh"),
+    "kt_min_max_swapped": ("e[0] = mn;\n                    e[1] = mx;", "e[0] = mx;\n                    e[1] = mn;"),
+    "score_min_corner_only": ("sh = sh + (lo > hi ? lo : hi);", "sh = sh + lo;"),
+    "score_last_head_only": ("total = total + sh;", "total = sh;"),
+    "ties_to_higher_page": ("if (best < 0 || s[p] > s[best])", "if (best < 0 || s[p] >= s[best])"),
+    "window_one_token_short": ("int lo = L - window > 0 ? L - window : 0;",
+                               "int lo = L - window + 1 > 0 ? L - window + 1 : 0;"),
+    "topk_one_short": ("for (int k = 0; k < topk; ++k) {", "for (int k = 1; k < topk; ++k) {"),
+    "sparse_last_token_dropped": ("int cnt = L - p * P < P ? L - p * P : P;",
+                                  "int cnt = L - p * P < P ? L - p * P - 1 : P;"),
 }
 
 
 def _pins():
     """Every pin, as zero-argument callables (parametrized ones expanded)."""
     fns = []
-    for mod, name in [(m, n) for m in (pins, append_pins) for n in dir(m)]:
+    for mod, name in [(m, n) for m in (pins, append_pins, sparse_pins) for n in dir(m)]:
         if not name.startswith("test_"):
             continue
         f = getattr(mod, name)
