@@ -395,6 +395,10 @@ def parse(argv=None):
     ap.add_argument("--append", action="store_true",
                     help="decode workloads: time gqa_paged_append_decode (each step first "
                          "writes the new token's K/V into its page)")
+    ap.add_argument("--sweep", default=None, choices=["config3", "splits"],
+                    help="print one JSON document of a decode sweep instead of the bench line: "
+                         "config3 = B x PackGQA x num_splits at ctx 2048 (bf16, e4m3); "
+                         "splits = the split schedule's time per split count and (B, ctx)")
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "long70b"],
                     help="decode: the headline (paged GQA decode); prefill: causal chunked "
                          "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]; "
@@ -731,6 +735,120 @@ def measure_decode(a, dev, rank, world, dist, with_cpu):
     }
 
 
+# ------------------------------------------------------------------------ sweeps
+
+L2_BYTES = 126 << 20
+
+
+def device_decode_inputs(B, ctx, Hq, Hk, D, P, kv, dev, seed, min_bytes=3 * L2_BYTES):
+    """Timing-only decode inputs made on the device (their values are N(0,1); parity is
+    the tests' job): a shuffled pool holding `copies` disjoint copies of the batch, so
+    that consecutive steps read different pages and the KV they touch (at least
+    min_bytes over the copies) does not sit in L2.  Returns (q, k, v, ks, vs, tables,
+    seq_lens, step_bytes)."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(seed)
+    npg = (ctx + P - 1) // P
+    elem = 1 if kv == "fp8_e4m3" else 2
+    kv_bytes = 2 * B * ctx * Hk * D * elem
+    copies = max(1, -(-min_bytes // max(kv_bytes, 1)))
+    used = B * npg * copies
+    pool = -(-used * 4 // 3)
+    perm = torch.randperm(pool, device=dev, generator=g).to(torch.int32)
+    tables = [perm[c * B * npg:(c + 1) * B * npg].view(B, npg).contiguous() for c in range(copies)]
+    k = torch.randn(pool, Hk, P, D, device=dev, generator=g, dtype=torch.bfloat16)
+    v = torch.randn(pool, Hk, P, D, device=dev, generator=g, dtype=torch.bfloat16)
+    ks = vs = None
+    if elem == 1:
+        def q8(x):
+            amax = x.float().abs().amax(dim=(2, 3))
+            sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+            y = (x.float() / sc[:, :, None, None]).clamp(-448.0, 448.0)
+            return y.to(torch.float8_e4m3fn).view(torch.uint8), sc.float().contiguous()
+        k, ks = q8(k)
+        v, vs = q8(v)
+    q = torch.randn(B, Hq, D, device=dev, generator=g, dtype=torch.bfloat16)
+    sl = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    return q, k, v, ks, vs, tables, sl, decode_step_bytes([ctx] * B, Hq, Hk, D, elem, P)
+
+
+def sweep_point(binding, inp, S, pack, dev, K=20, repeat_s=0.25):
+    """GB/s of one decode configuration: K steps (each on the next copy of the batch) as a
+    CUDA graph, median of repeated replays."""
+    import torch
+    q, k, v, ks, vs, tables, sl, step_bytes = inp
+    B, Hq, D = q.shape
+    num_pages, Hk, P, _ = k.shape
+    kvc = binding.GQA_KV_FP8_E4M3 if ks is not None else binding.GQA_KV_BF16
+    pts = tables[0].shape[1]
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ws = binding.new_workspace(binding.gqa_paged_decode_workspace_size(B, Hq, Hk, D, P, pts * P,
+                                                                       kvc, S), dev)
+    stream = torch.cuda.current_stream(dev)
+    K = max(K, len(tables))
+    it = [0]
+
+    def step(on):
+        t = tables[it[0] % len(tables)]
+        it[0] += 1
+        binding.gqa_paged_decode(q, k, v, t, sl, 1.0 / math.sqrt(D), num_splits=S, pack_gqa=pack,
+                                 k_scale=ks, v_scale=vs, out=out, lse=lse, workspace=ws, stream=on)
+
+    for _ in range(3):
+        step(stream)
+    torch.cuda.synchronize(dev)
+    assert binding.gqa_get_error(ws) == 0
+    ms, sp = timed_graph(step, K, stream, dev, repeat_s)
+    med = sp["median_ms"] if sp else ms
+    return {"ms": round(med, 5), "us": round(med * 1e3, 2),
+            "gbs": round(step_bytes / (med * 1e-3) / 1e9, 1),
+            "pct_of_hbm_peak": round(100 * step_bytes / (med * 1e-3) / 1e9 / peaks()[0], 2),
+            "copies": len(tables)}
+
+
+def run_sweep(kind, a, dev):
+    """config3: the batch-sensitivity grid (Hq=32, Hk=8, D=128, ctx 2048, page 16):
+    B x PackGQA on/off x num_splits {1, 2, 4, auto}, bf16 and e4m3 KV.
+    splits: the split schedule's best split count per (batch, context), the table
+    gqa_pick_splits encodes."""
+    import torch
+    from gqa_attention_paged_b200 import binding
+    Hq, Hk, D, P = 32, 8, 128, 16
+    res = {"kind": kind, "peak_gbs": peaks()[0], "points": []}
+    if kind == "config3":
+        for kv in ("bf16", "fp8_e4m3"):
+            for B in (1, 16, 32, 64, 128, 256):
+                inp = device_decode_inputs(B, 2048, Hq, Hk, D, P, kv, dev, seed=B)
+                for pack in (True, False):
+                    for S in (1, 2, 4, 0):
+                        if kv == "fp8_e4m3" and not pack and S != 0:
+                            continue
+                        r = sweep_point(binding, inp, S, pack, dev)
+                        r.update({"B": B, "ctx": 2048, "kv": kv, "pack_gqa": pack,
+                                  "num_splits": "auto" if S == 0 else S})
+                        res["points"].append(r)
+                        print(json.dumps(r), file=sys.stderr, flush=True)
+                del inp
+                torch.cuda.empty_cache()
+    else:
+        grid = [(1, 512), (1, 2048), (1, 8192), (1, 32768), (4, 2048), (4, 8192), (4, 32768),
+                (16, 512), (16, 2048), (16, 8192), (16, 32768), (64, 512), (64, 2048),
+                (64, 8192), (256, 512), (256, 2048), (1024, 512), (1024, 1024)]
+        for B, ctx in grid:
+            inp = device_decode_inputs(B, ctx, Hq, Hk, D, P, "bf16", dev, seed=B + ctx)
+            for S in (1, 2, 4, 8, 16, 32):
+                if S > (ctx // P):
+                    continue
+                r = sweep_point(binding, inp, S, True, dev)
+                r.update({"B": B, "ctx": ctx, "num_splits": S})
+                res["points"].append(r)
+                print(json.dumps(r), file=sys.stderr, flush=True)
+            del inp
+            torch.cuda.empty_cache()
+    return res
+
+
 def _secondary_summary(line):
     keep = ("metric", "value", "unit", "ms_per_step", "spread", "roofline", "clocks", "e2e",
             "cpu_baseline", "gpu_launches", "pct_of_hbm_peak", "pct_of_bf16_peak", "dtype")
@@ -758,6 +876,10 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
+    if a.sweep:
+        if rank == 0:
+            print(json.dumps(run_sweep(a.sweep, a, dev)))
+        return 0
     if a.workload == "prefill":
         if rank != 0:
             return 0

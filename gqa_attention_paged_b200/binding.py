@@ -36,6 +36,14 @@ SIGNATURES = {
                               ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
     "gqa_paged_decode_partial": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                       ctypes.c_float, _I, _I, _P, _P, _P, _SZ, _P]),
+    "gqa_paged_kt_build": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "gqa_paged_kt_append": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "gqa_paged_sparse_table_stride": (_I, [_I, _I, _I, _I]),
+    "gqa_paged_sparse_select": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+                                     _P, _P, _P, _P]),
+    "gqa_paged_sparse_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "gqa_paged_sparse_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                     ctypes.c_float, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "gqa_paged_decode_static_scratch": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
                                              _I, _I, _I, ctypes.c_float, _I, _I, _P, _P, _P]),
     "gqa_paged_prefill_workspace_size": (_SZ, [_I, _I, _I]),
@@ -439,3 +447,130 @@ def gqa_get_error(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise the stream, return and clear the device error word of `workspace`."""
     _need(workspace, "workspace", torch.uint8)
     return load().gqa_get_error(_ptr(workspace), _stream(stream))
+
+
+# ------------------------------------------------------------------------ sparse decode
+
+def _sparse_common(q, k_pages, page_table, seq_lens):
+    _need(q, "q", torch.bfloat16)
+    B, Hq, D = q.shape
+    _need(k_pages, "k_pages", torch.bfloat16)
+    num_pages, Hk, P, D2 = k_pages.shape
+    if D2 != D:
+        raise ValueError("head_dim of q and the KV pools differ")
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B][pt_stride]")
+    return B, Hq, Hk, D, P, num_pages, page_table.shape[1]
+
+
+def new_kt_cache(k_pages: torch.Tensor) -> torch.Tensor:
+    """An empty KT cache for a bf16 pool: bf16 [num_pages][Hk][D][2]."""
+    num_pages, Hk, P, D = k_pages.shape
+    return torch.zeros(num_pages, Hk, D, 2, dtype=torch.bfloat16, device=k_pages.device)
+
+
+def gqa_paged_kt_build(k_pages: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
+                       kt: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """KT entries (per page and kv head: min and max of the keys over the valid tokens)
+    of every page the sequences reference; returns kt bf16 [num_pages][Hk][D][2]."""
+    _need(k_pages, "k_pages", torch.bfloat16)
+    num_pages, Hk, P, D = k_pages.shape
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32)
+    B = seq_lens.shape[0]
+    if kt is None:
+        kt = new_kt_cache(k_pages)
+    _need(kt, "kt", torch.bfloat16, (num_pages, Hk, D, 2))
+    if workspace is None:
+        workspace = new_workspace(256, k_pages.device)
+    st = load().gqa_paged_kt_build(_ptr(k_pages), _ptr(page_table), page_table.shape[1],
+                                   _ptr(seq_lens), B, Hk, D, P, num_pages, _ptr(kt),
+                                   _ptr(workspace), _stream(stream))
+    _check("gqa_paged_kt_build", st)
+    return kt
+
+
+def gqa_paged_kt_append(k_new: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
+                        kt: torch.Tensor, page_size: int,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Update the KT entries with the token at position seq_lens[b] - 1 (k_new bf16
+    [B][Hk][D]), in place."""
+    _need(k_new, "k_new", torch.bfloat16)
+    B, Hk, D = k_new.shape
+    _need(kt, "kt", torch.bfloat16)
+    num_pages = kt.shape[0]
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if workspace is None:
+        workspace = new_workspace(256, kt.device)
+    st = load().gqa_paged_kt_append(_ptr(k_new), _ptr(page_table), page_table.shape[1],
+                                    _ptr(seq_lens), B, Hk, D, int(page_size), num_pages, _ptr(kt),
+                                    _ptr(workspace), _stream(stream))
+    _check("gqa_paged_kt_append", st)
+    return kt
+
+
+def gqa_paged_sparse_table_stride(pt_stride: int, page_size: int, topk: int, window: int) -> int:
+    return load().gqa_paged_sparse_table_stride(pt_stride, page_size, topk, window)
+
+
+def gqa_paged_sparse_select(q: torch.Tensor, kt: torch.Tensor, k_pages: torch.Tensor,
+                            page_table: torch.Tensor, seq_lens: torch.Tensor, topk: int,
+                            window: int, workspace: Optional[torch.Tensor] = None,
+                            stream=None):
+    """The chosen pages: returns (sel_table int32 [B*Hk][ss] of physical*Hk + kv head,
+    sel_lens int32 [B*Hk], sel_pages int32 [B*Hk][ss] logical pages)."""
+    B, Hq, Hk, D, P, num_pages, pts = _sparse_common(q, k_pages, page_table, seq_lens)
+    _need(kt, "kt", torch.bfloat16, (num_pages, Hk, D, 2))
+    ss = gqa_paged_sparse_table_stride(pts, P, topk, window)
+    dev = q.device
+    sel_table = torch.full((B * Hk, max(ss, 1)), -1, dtype=torch.int32, device=dev)
+    sel_pages = torch.full((B * Hk, max(ss, 1)), -1, dtype=torch.int32, device=dev)
+    sel_lens = torch.zeros(B * Hk, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(256, dev)
+    st = load().gqa_paged_sparse_select(_ptr(q), _ptr(kt), _ptr(page_table), pts, _ptr(seq_lens),
+                                        B, Hq, Hk, D, P, num_pages, int(topk), int(window),
+                                        _ptr(sel_table), max(ss, 1), _ptr(sel_lens),
+                                        _ptr(sel_pages), _ptr(workspace), _stream(stream))
+    _check("gqa_paged_sparse_select", st)
+    return sel_table, sel_lens, sel_pages
+
+
+def gqa_paged_sparse_decode_workspace_size(B, Hq, Hk, head_dim, page_size, pt_stride, topk,
+                                           window, num_splits=0) -> int:
+    return load().gqa_paged_sparse_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                         pt_stride, topk, window, num_splits)
+
+
+def gqa_paged_sparse_decode(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                            kt: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
+                            scale: float, topk: int, window: int, num_splits: int = 0,
+                            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None, want_lse: bool = True,
+                            stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Page-level top-K sparse decode (bf16 pools): the window pages plus the topk
+    best-scoring earlier pages of every (sequence, kv head) are attended."""
+    B, Hq, Hk, D, P, num_pages, pts = _sparse_common(q, k_pages, page_table, seq_lens)
+    _need(v_pages, "v_pages", torch.bfloat16, k_pages.shape)
+    _need(kt, "kt", torch.bfloat16, (num_pages, Hk, D, 2))
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq))
+    need = gqa_paged_sparse_decode_workspace_size(B, Hq, Hk, D, P, pts, topk, window, num_splits)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = load().gqa_paged_sparse_decode(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kt), _ptr(page_table), pts, _ptr(seq_lens),
+        B, Hq, Hk, D, P, num_pages, float(scale), int(topk), int(window), int(num_splits),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("gqa_paged_sparse_decode", st)
+    return out, lse

@@ -302,7 +302,7 @@ int gqa_paged_prefill(const void *q, const int32_t *cu_q, const void *k_pages,
     if (!q || !cu_q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !workspace)
         return GQA_ERR_NULL;
     if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || Hk > 65535 ||
-        Hq / Hk > 128 || head_dim != 128 || !valid_page_size(page_size) || num_pages <= 0 ||
+        Hq / Hk > 128 || (head_dim != 64 && head_dim != 128) || !valid_page_size(page_size) || num_pages <= 0 ||
         pt_stride <= 0 || total_q < 0 || max_q_len < 0 || !(scale > 0.f) ||
         (int64_t)num_pages * Hk * page_size > INT32_MAX ||
         (int64_t)pt_stride * page_size > INT32_MAX)
@@ -451,6 +451,129 @@ int gqa_paged_append_decode(const void *q, const void *k_new, const void *v_new,
                             pt_stride, seq_lens, B, Hq, Hk, head_dim, page_size, num_pages,
                             scale, num_splits, pack_gqa, out, lse, workspace, workspace_bytes,
                             stream);
+}
+
+int gqa_paged_kt_build(const void *k_pages, const int32_t *page_table, int pt_stride,
+                       const int32_t *seq_lens, int B, int Hk, int head_dim, int page_size,
+                       int num_pages, void *kt, void *workspace, cudaStream_t stream) {
+    if (!k_pages || !page_table || !seq_lens || !kt || !workspace) return GQA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hk <= 0 || (head_dim != 64 && head_dim != 128) ||
+        !valid_page_size(page_size) || num_pages <= 0 || pt_stride <= 0 ||
+        (int64_t)num_pages * Hk * page_size > INT32_MAX || (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (!aligned(k_pages, 16) || !aligned(kt, 16) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(workspace, 256))
+        return GQA_ERR_ALIGN;
+    return launch_kt_build(k_pages, page_table, pt_stride, seq_lens, B, Hk, head_dim, page_size,
+                           num_pages, kt, static_cast<int *>(workspace), stream) == cudaSuccess
+               ? GQA_OK
+               : GQA_ERR_LAUNCH;
+}
+
+int gqa_paged_kt_append(const void *k_new, const int32_t *page_table, int pt_stride,
+                        const int32_t *seq_lens, int B, int Hk, int head_dim, int page_size,
+                        int num_pages, void *kt, void *workspace, cudaStream_t stream) {
+    if (!k_new || !page_table || !seq_lens || !kt || !workspace) return GQA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hk <= 0 || (head_dim != 64 && head_dim != 128) ||
+        !valid_page_size(page_size) || num_pages <= 0 || pt_stride <= 0 ||
+        (int64_t)num_pages * Hk * page_size > INT32_MAX || (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (!aligned(k_new, 2) || !aligned(kt, 16) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(workspace, 256))
+        return GQA_ERR_ALIGN;
+    return launch_kt_append(k_new, page_table, pt_stride, seq_lens, B, Hk, head_dim, page_size,
+                            num_pages, kt, static_cast<int *>(workspace), stream) == cudaSuccess
+               ? GQA_OK
+               : GQA_ERR_LAUNCH;
+}
+
+int gqa_paged_sparse_table_stride(int pt_stride, int page_size, int topk, int window) {
+    if (pt_stride <= 0 || page_size <= 0 || topk < 0 || window < 0) return 0;
+    // topk earlier pages plus the pages a window of `window` tokens can touch
+    const int64_t win_pages = window > 0 ? ((int64_t)window + page_size - 1) / page_size + 1 : 0;
+    const int64_t s = (int64_t)topk + win_pages;
+    return (int)(s < pt_stride ? s : pt_stride);
+}
+
+int gqa_paged_sparse_select(const void *q, const void *kt, const int32_t *page_table,
+                            int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
+                            int head_dim, int page_size, int num_pages, int topk, int window,
+                            int32_t *sel_table, int sel_stride, int32_t *sel_lens,
+                            int32_t *sel_pages, void *workspace, cudaStream_t stream) {
+    if (!q || !kt || !page_table || !seq_lens || !sel_table || !sel_lens || !workspace)
+        return GQA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 ||
+        Hq / Hk > kSparseMaxGroup || (head_dim != 64 && head_dim != 128) ||
+        !valid_page_size(page_size) || num_pages <= 0 || pt_stride <= 0 ||
+        pt_stride > kSparseMaxPages || topk < 0 || window < 0 ||
+        sel_stride < gqa_paged_sparse_table_stride(pt_stride, page_size, topk, window) ||
+        (int64_t)num_pages * Hk * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(kt, 16) || !aligned(page_table, 4) || !aligned(seq_lens, 4) ||
+        !aligned(sel_table, 4) || !aligned(sel_lens, 4) || (sel_pages && !aligned(sel_pages, 4)) ||
+        !aligned(workspace, 256))
+        return GQA_ERR_ALIGN;
+    return launch_sparse_select(q, kt, page_table, pt_stride, seq_lens, B, Hq, Hk, head_dim,
+                                page_size, num_pages, topk, window, sel_table, sel_stride,
+                                sel_lens, sel_pages, static_cast<int *>(workspace), stream) ==
+                   cudaSuccess
+               ? GQA_OK
+               : GQA_ERR_LAUNCH;
+}
+
+size_t gqa_paged_sparse_decode_workspace_size(int B, int Hq, int Hk, int head_dim,
+                                              int page_size, int pt_stride, int topk, int window,
+                                              int num_splits) {
+    if (B < 0 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0) return 0;
+    const int ss = gqa_paged_sparse_table_stride(pt_stride, page_size, topk, window);
+    if (ss <= 0) return 0;
+    const int Bv = B * Hk;
+    return gqa_paged_decode_workspace_size(Bv, Hq / Hk, 1, head_dim, page_size, ss * page_size,
+                                           GQA_KV_BF16, num_splits) +
+           align_up((size_t)Bv * sizeof(int32_t), 256) +
+           align_up((size_t)Bv * ss * sizeof(int32_t), 256);
+}
+
+int gqa_paged_sparse_decode(const void *q, const void *k_pages, const void *v_pages,
+                            const void *kt, const int32_t *page_table, int pt_stride,
+                            const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim,
+                            int page_size, int num_pages, float scale, int topk, int window,
+                            int num_splits, void *out, float *lse, void *workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+    if (!q || !k_pages || !v_pages || !kt || !page_table || !seq_lens || !out || !workspace)
+        return GQA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 ||
+        Hq / Hk > kSparseMaxGroup || (head_dim != 64 && head_dim != 128) ||
+        !valid_page_size(page_size) || num_pages <= 0 || pt_stride <= 0 ||
+        pt_stride > kSparseMaxPages || topk < 0 || window < 0 ||
+        (int64_t)B * Hk > 65535 || (int64_t)num_pages * Hk * page_size > INT32_MAX ||
+        (int64_t)pt_stride * page_size > INT32_MAX)
+        return GQA_ERR_SHAPE;
+    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(kt, 16) ||
+        !aligned(out, 16) || !aligned(page_table, 4) || !aligned(seq_lens, 4) ||
+        (lse && !aligned(lse, 4)))
+        return GQA_ERR_ALIGN;
+    const size_t need = gqa_paged_sparse_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
+                                                               pt_stride, topk, window, num_splits);
+    if (!aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
+    if (B == 0) return GQA_OK;
+    const int ss = gqa_paged_sparse_table_stride(pt_stride, page_size, topk, window);
+    const int Bv = B * Hk, g = Hq / Hk;
+    const size_t dws = gqa_paged_decode_workspace_size(Bv, g, 1, head_dim, page_size,
+                                                       ss * page_size, GQA_KV_BF16, num_splits);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int32_t *sel_lens = reinterpret_cast<int32_t *>(ws + dws);
+    int32_t *sel_table = reinterpret_cast<int32_t *>(ws + dws + align_up((size_t)Bv * 4, 256));
+    if (launch_sparse_select(q, kt, page_table, pt_stride, seq_lens, B, Hq, Hk, head_dim,
+                             page_size, num_pages, topk, window, sel_table, ss, sel_lens, nullptr,
+                             reinterpret_cast<int *>(ws), stream) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    // the chosen pages of every (sequence, kv head) as one sequence of a decode with one kv
+    // head: q [B*Hk][g][D], pools [num_pages*Hk][1][P][D], out [B*Hk][g][D]
+    return decode_call(q, k_pages, v_pages, nullptr, nullptr, GQA_KV_BF16, sel_table, ss,
+                       sel_lens, Bv, g, 1, head_dim, page_size, num_pages * Hk, scale,
+                       num_splits, 1, out, 0, lse, workspace, dws, stream);
 }
 
 int gqa_get_error(void *workspace, cudaStream_t stream) {

@@ -134,6 +134,23 @@ struct AppendArgs {
 };
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t stream);
 
+// Page-level top-K sparse decode (sparse.cu).  KT cache: bf16 [num_pages][Hk][D][2].
+cudaError_t launch_kt_build(const void *k_pages, const int32_t *page_table, int pt_stride,
+                            const int32_t *seq_lens, int B, int Hk, int D, int P, int num_pages,
+                            void *kt, int *err, cudaStream_t stream);
+cudaError_t launch_kt_append(const void *k_new, const int32_t *page_table, int pt_stride,
+                             const int32_t *seq_lens, int B, int Hk, int D, int P, int num_pages,
+                             void *kt, int *err, cudaStream_t stream);
+size_t sparse_select_smem_bytes(int g, int D, int pt_stride);
+cudaError_t launch_sparse_select(const void *q, const void *kt, const int32_t *page_table,
+                                 int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
+                                 int D, int P, int num_pages, int topk, int window,
+                                 int32_t *sel_table, int sel_stride, int32_t *sel_lens,
+                                 int32_t *sel_pages, int *err, cudaStream_t stream);
+// Largest page table (pages per sequence) and group the sparse selection takes.
+constexpr int kSparseMaxPages = 16384;
+constexpr int kSparseMaxGroup = 16;
+
 // Tokens per decode pipeline stage (the TMA box height of the KV tensor maps): 32 for
 // e4m3 KV on pages of at least 32 tokens, else 16.
 inline int decode_tile_tokens(int kv_dtype, int page_size) {

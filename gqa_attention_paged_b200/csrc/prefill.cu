@@ -45,12 +45,13 @@ namespace {
 constexpr int kM = 128;                // packed query rows per query tile
 constexpr int kQT = 2;                 // query tiles per CTA
 constexpr int kN = 128;                // keys per KV tile
-constexpr int kD = 128;                // head dim
 constexpr int kKStages = 2;            // K ring depth
 constexpr int kVStages = 3;            // V ring depth (a V tile also waits for its conversion)
 constexpr int kThreadsP = 384;
 constexpr int kHalfBytes = kM * 128;   // one 64-column (128-byte) half of a 128-row tile
-constexpr int kTileBytesP = 2 * kHalfBytes;
+// A 128-row tile of head dim D: D / 64 halves.
+template <int D>
+__host__ __device__ constexpr int tile_bytes() { return (D / 64) * kHalfBytes; }
 constexpr int kChunk = 16;             // keys per TMA copy (one box)
 constexpr int kChunkBytes = kChunk * 128;
 constexpr float kLog2eP = 1.4426950408889634f;
@@ -66,10 +67,11 @@ constexpr int kConvThreads = 64;
 // |bf16 bits| at or above this (2^16, and Inf / NaN) does not convert to a finite f16
 constexpr uint32_t kF16Limit = 0x4780u;
 
+template <int D>
 struct alignas(1024) PSmem {
-    uint8_t q[kQT][kTileBytesP];
-    uint8_t k[kKStages][kTileBytesP];
-    uint8_t v[kVStages][kTileBytesP];
+    uint8_t q[kQT][tile_bytes<D>()];
+    uint8_t k[kKStages][tile_bytes<D>()];
+    uint8_t v[kVStages][tile_bytes<D>()];
     uint64_t q_full;
     uint64_t k_full[kKStages], k_empty[kKStages];
     uint64_t v_full[kVStages], v_ready[kVStages], v_empty[kVStages];
@@ -80,7 +82,7 @@ struct alignas(1024) PSmem {
     uint32_t tmem_base;
 };
 
-static_assert(sizeof(PSmem) + 1024 <= 227 * 1024, "shared memory per CTA");
+static_assert(sizeof(PSmem<128>) + 1024 <= 227 * 1024, "shared memory per CTA");
 
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);
@@ -104,7 +106,8 @@ __device__ __forceinline__ int kv_chunk_row(const PrefillArgs &a, const int32_t 
 
 // Softmax warpgroup of query tile (warp - 4) / 4: online softmax over the score tiles in
 // tensor memory, P written back over S, final O / l and LSE to global memory.
-__device__ __forceinline__ void softmax_role(PSmem &sm, const PrefillArgs &a, const uint32_t tmem,
+template <int D>
+__device__ __forceinline__ void softmax_role(PSmem<D> &sm, const PrefillArgs &a, const uint32_t tmem,
                                              const int warp, const int lane, const int (&n_kv_q)[kQT],
                                              const int b, const int kvh, const int g, const int q0,
                                              const int Lq, const int i0, const int T, const int L) {
@@ -171,7 +174,7 @@ __device__ __forceinline__ void softmax_role(PSmem &sm, const PrefillArgs &a, co
             }
             tc_fence_after_sync();
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
                 tmem_ld32(tO + 32 * cc, o);
                 tmem_wait_ld();
@@ -256,9 +259,9 @@ __device__ __forceinline__ void softmax_role(PSmem &sm, const PrefillArgs &a, co
         tc_fence_after_sync();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.out) +
-                             ((size_t)(q0 + tok) * a.Hq + kvh * g + hh) * kD;
+                             ((size_t)(q0 + tok) * a.Hq + kvh * g + hh) * D;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + 32 * cc, o);
             tmem_wait_ld();
@@ -342,12 +345,14 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreadsP, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                    const __grid_constant__ CUtensorMap qmap, const PrefillArgs a, const int T) {
     extern __shared__ uint8_t smem_raw[];
-    PSmem &sm = *reinterpret_cast<PSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+    constexpr int kHalves = D / 64;
+    PSmem<D> &sm = *reinterpret_cast<PSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                 ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // block i = (work item i / Hk in the plan's longest-first order, kv head i % Hk), so
     // the longest items are dispatched first, all heads of an item together
@@ -410,7 +415,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 
     if (warp >= 4) {
         regs_acquire<kRegsSoftmax>();
-        softmax_role(sm, a, tmem, warp, lane, n_kv_q, b, kvh, g, q0, Lq, i0, T, L);
+        softmax_role<D>(sm, a, tmem, warp, lane, n_kv_q, b, kvh, g, q0, Lq, i0, T, L);
     } else {
     // every warp of warpgroup 0 gives its registers back at the same instruction
     regs_release<kRegsSide>();
@@ -421,9 +426,9 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             prefetch_tensormap(&qmap);
             prefetch_tensormap(&kmap);
             prefetch_tensormap(&vmap);
-            mbar_arrive_expect_tx(&sm.q_full, kQT * 2 * g * T * 128);
+            mbar_arrive_expect_tx(&sm.q_full, kQT * kHalves * g * T * 128);
             for (int q = 0; q < kQT; ++q)
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < kHalves; ++h)
                     tma_load_3d(sm.q[q] + h * kHalfBytes, &qmap, &sm.q_full, 64 * h, kvh * g,
                                 q0 + i0 + q * T, policy_evict_first());
         }
@@ -439,13 +444,13 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     set_error(a.err, GQA_ERR_TIMEOUT);
                     fail = true;
                 } else {
-                    mbar_arrive_expect_tx(&sm.k_full[ks], __popc(mask) * 2 * kChunkBytes);
+                    mbar_arrive_expect_tx(&sm.k_full[ks], __popc(mask) * kHalves * kChunkBytes);
                 }
             }
             if (__shfl_sync(kAll, fail, 0)) break;
             if (row >= 0) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < kHalves; ++h)
                     tma_load_2d(sm.k[ks] + h * kHalfBytes + lane * kChunkBytes, &kmap,
                                 &sm.k_full[ks], 64 * h, row, pol_kv);
             }
@@ -463,8 +468,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);   // Q, K both K-major
-        constexpr uint32_t idesc_pv16 = idesc_f16_f32(kM, kD, 0, 1);  // P (TMEM), V MN-major
-        constexpr uint32_t idesc_pvbf = idesc_bf16_f32(kM, kD, 0, 1);
+        constexpr uint32_t idesc_pv16 = idesc_f16_f32(kM, D, 0, 1);  // P (TMEM), V MN-major
+        constexpr uint32_t idesc_pvbf = idesc_bf16_f32(kM, D, 0, 1);
         bool ok = wait_all(&sm.q_full, 0);
         // S_q(j) = Q_q K_j^T into tensor-memory columns [128 q, 128 q + 128)
         auto issue_s = [&](int q, int j) -> bool {
@@ -474,7 +479,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             if (lane == 0) {
                 const uint32_t qa = smem_u32(sm.q[q]), ka = smem_u32(sm.k[stage]);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
                     tc_mma_ss(tmem + 128 * q, smem_desc_sw128(qa + off, 16, 1024),
                               smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
@@ -543,7 +548,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         // that tile's stage and loads tile j + kVStages - 1 into it.
         const int cid = threadIdx.x - 64;  // 0..63
         const int cw = warp - 2;
-        constexpr int kChunks16 = kTileBytesP / 16;  // 16-byte chunks of a V tile
+        constexpr int kChunks16 = tile_bytes<D>() / 16;  // 16-byte chunks of a V tile
         const int32_t *pt = a.page_table + (size_t)b * a.pt_stride;
         const uint64_t pol_kv = policy_evict_last();
         int issued_v = 0;
@@ -551,11 +556,11 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             const int row = kv_chunk_row(a, pt, jv, lane, kvh, L);
             const unsigned mask = __ballot_sync(kAll, row >= 0);
             const int vs = jv % kVStages;
-            if (lane == 0) mbar_arrive_expect_tx(&sm.v_full[vs], __popc(mask) * 2 * kChunkBytes);
+            if (lane == 0) mbar_arrive_expect_tx(&sm.v_full[vs], __popc(mask) * kHalves * kChunkBytes);
             __syncwarp();
             if (row >= 0) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < kHalves; ++h)
                     tma_load_2d(sm.v[vs] + h * kHalfBytes + lane * kChunkBytes, &vmap,
                                 &sm.v_full[vs], 64 * h, row, pol_kv);
             }
@@ -664,22 +669,29 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     }
 }
 
-}  // namespace
-
-cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
-                           const CUtensorMap &qmap, cudaStream_t stream) {
+template <int D>
+cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                             const CUtensorMap &qmap, cudaStream_t stream) {
     const int g = a.Hq / a.Hk;
     const int T = kM / g;
-    const size_t smem = sizeof(PSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = sizeof(PSmem<D>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int items_per_seq = (a.max_q_len + kQT * T - 1) / (kQT * T);
     if (items_per_seq == 0 || a.B == 0) return cudaSuccess;
     prefill_plan_kernel<<<1, 1024, 0, stream>>>(a, T, items_per_seq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    prefill_kernel<<<a.B * items_per_seq * a.Hk, kThreadsP, smem, stream>>>(kmap, vmap, qmap, a, T);
+    prefill_kernel<D><<<a.B * items_per_seq * a.Hk, kThreadsP, smem, stream>>>(kmap, vmap, qmap, a, T);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                           const CUtensorMap &qmap, cudaStream_t stream) {
+    return a.D == 64 ? launch_prefill_d<64>(a, kmap, vmap, qmap, stream)
+                     : launch_prefill_d<128>(a, kmap, vmap, qmap, stream);
 }
 
 }  // namespace gqa

@@ -247,7 +247,7 @@ size_t gqa_paged_prefill_workspace_size(int total_q, int Hq, int head_dim);
  *   cu_q       int32 [B+1], cu_q[0] = 0, nondecreasing, cu_q[B] = total_q,
  *              cu_q[b+1] - cu_q[b] <= max_q_len and <= seq_lens[b]
  *   k_pages, v_pages, page_table, pt_stride, seq_lens: as for decode (bf16 KV only)
- *   head_dim   128; page_size in {16, 32, 64}; Hq / Hk <= 128; scale > 0
+ *   head_dim   64 or 128; page_size in {16, 32, 64}; Hq / Hk <= 128; scale > 0
  *   out        bf16 [total_q][Hq][head_dim];  lse fp32 [total_q][Hq] or NULL
  *   workspace  >= gqa_paged_prefill_workspace_size(...) bytes, zeroed before first use
  */
@@ -326,6 +326,95 @@ int gqa_paged_gather(const void *k_pages, const void *v_pages, const int32_t *pa
                      int pt_stride, const int32_t *seq_lens, const int64_t *cu_kv, int B,
                      int Hk, int head_dim, int page_size, int num_pages, int elem_bytes,
                      void *k_out, void *v_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Page-level top-K sparse decode: the decode stage of RocketKV as
+ * "TensorRT-LLM 如何用 sparse_attention_config 配置 Sparse Attention 降低长上下文推理开销"
+ * (RocketKV configuration section) configures it: an auxiliary KT cache scores every page
+ * of a sequence, and the decode attends to the `topk` best pages plus the pages holding the
+ * last `window` tokens (the page's window_size), skipping the rest.  The page leaves the
+ * KT cache and the score unstated; this library reads them as follows.
+ *   - KT entry of (page, kv head): the element-wise minimum and maximum of the page's key
+ *     vectors over its valid tokens.  kt: bf16 [num_pages][Hk][head_dim][2], (min, max)
+ *     per dim, 16-byte aligned, owned by the caller (like the KV pools).
+ *   - Score of a page for kv head j: over the g query heads h of the group,
+ *     sum_h sum_d max(q[h][d] * min_d, q[h][d] * max_d), the largest q.k over the box
+ *     [min, max] (an upper bound of q.k for every key of the page).  fp32, d ascending
+ *     per head, then heads ascending (every product of two bf16 values is exact in fp32).
+ *   - Selection per (sequence, kv head): the pages holding any of the last `window` tokens
+ *     (none when window = 0), plus the `topk` highest-scoring earlier pages, equal scores
+ *     going to the lower logical page; all earlier pages when there are at most `topk`.
+ *     The selection unit is one cache page (the page's sparse page_size, a power of two,
+ *     taken equal to page_size), and every query channel is used (the page's topr =
+ *     head_dim).
+ *   - Attention: softmax attention of every query head over the tokens of its kv head's
+ *     chosen pages, computed by the decode kernels of gqa_paged_decode().
+ * bf16 pools only; head_dim in {64, 128}; Hq / Hk <= 16; pt_stride <= 16384.
+ * ------------------------------------------------------------------------------------- */
+
+/*
+ * KT entries of every page the sequences reference: for sequence b and logical page
+ * p < ceil(seq_lens[b] / page_size), the min / max over the page's
+ * min(page_size, seq_lens[b] - p * page_size) valid tokens.  Entries of unreferenced pages
+ * are not written.  A page referenced by several sequences must hold the same number of
+ * valid tokens in each (shared prefix pages are full pages); they then write equal values.
+ * workspace: >= 256 bytes, 256-byte aligned; its error word records page-table entries or
+ * sequence lengths out of range.
+ */
+int gqa_paged_kt_build(const void *k_pages, const int32_t *page_table, int pt_stride,
+                       const int32_t *seq_lens, int B, int Hk, int head_dim, int page_size,
+                       int num_pages, void *kt, void *workspace, cudaStream_t stream);
+
+/*
+ * KT update for the token gqa_paged_append_kv() writes (position seq_lens[b] - 1): a token
+ * that opens a page (slot 0) sets the page's entry to (k, k), a later one takes the
+ * element-wise min / max with it.  k_new bf16 [B][Hk][head_dim].  After appends, the
+ * entries equal gqa_paged_kt_build()'s for the grown sequences.
+ */
+int gqa_paged_kt_append(const void *k_new, const int32_t *page_table, int pt_stride,
+                        const int32_t *seq_lens, int B, int Hk, int head_dim, int page_size,
+                        int num_pages, void *kt, void *workspace, cudaStream_t stream);
+
+/*
+ * Entries per row of the chosen-page table: min(pt_stride, topk + window pages), the
+ * window touching at most ceil(window / page_size) + 1 pages.  0 for invalid arguments.
+ */
+int gqa_paged_sparse_table_stride(int pt_stride, int page_size, int topk, int window);
+
+/*
+ * The selection alone.  For row r = b * Hk + j (sequence b, kv head j):
+ *   sel_table int32 [B*Hk][sel_stride]: the chosen pages in ascending logical order, each
+ *             as physical page * Hk + j (the (page, kv head) block's index when the pools
+ *             are seen as [num_pages * Hk][1][page_size][head_dim])
+ *   sel_lens  int32 [B*Hk]: tokens in the chosen pages
+ *   sel_pages int32 [B*Hk][sel_stride] or NULL: the chosen logical page indices
+ *   sel_stride >= gqa_paged_sparse_table_stride(pt_stride, page_size, topk, window)
+ * workspace: >= 256 bytes, 256-byte aligned (error word).
+ */
+int gqa_paged_sparse_select(const void *q, const void *kt, const int32_t *page_table,
+                            int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
+                            int head_dim, int page_size, int num_pages, int topk, int window,
+                            int32_t *sel_table, int sel_stride, int32_t *sel_lens,
+                            int32_t *sel_pages, void *workspace, cudaStream_t stream);
+
+/* Workspace of gqa_paged_sparse_decode(): the decode's for B*Hk sequences of one kv head
+ * and g = Hq/Hk heads, then the chosen-page lengths and table. */
+size_t gqa_paged_sparse_decode_workspace_size(int B, int Hq, int Hk, int head_dim,
+                                              int page_size, int pt_stride, int topk, int window,
+                                              int num_splits);
+
+/*
+ * Sparse decode: the selection, then the decode over the chosen pages, on `stream`.
+ * q, pools, page_table, seq_lens, scale, num_splits, out, lse as for gqa_paged_decode()
+ * (bf16 pools); kt as for gqa_paged_kt_build(); B * Hk <= 65535.  The workspace holds the
+ * chosen-page table between the two kernels; zero it once before first use.
+ */
+int gqa_paged_sparse_decode(const void *q, const void *k_pages, const void *v_pages,
+                            const void *kt, const int32_t *page_table, int pt_stride,
+                            const int32_t *seq_lens, int B, int Hq, int Hk, int head_dim,
+                            int page_size, int num_pages, float scale, int topk, int window,
+                            int num_splits, void *out, float *lse, void *workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Synchronises `stream`, returns the device error word held in `workspace`

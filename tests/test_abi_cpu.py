@@ -145,7 +145,8 @@ def test_prefill_rejects_bad_arguments_on_the_host():
         args.update(kw)
         return lib.gqa_paged_prefill(*args.values())
     assert call(q=None) == -1
-    assert call(D=64) == -2
+    assert call(D=96) == -2
+    assert call(D=256) == -2
     assert call(scale=0.0) == -2
     assert call(scale=-1.0) == -2
     assert call(Hq=6, Hk=4) == -2

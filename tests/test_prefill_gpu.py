@@ -47,6 +47,16 @@ def test_prefill_group_sizes_and_pages(Hq, Hk, P):
     check(out, lse, ref_o, ref_l, f"Hq={Hq} Hk={Hk} P={P}")
 
 
+@pytest.mark.parametrize("Hq,Hk,P,causal", [(8, 2, 16, True), (32, 8, 16, True),
+                                            (16, 16, 32, True), (8, 1, 64, False)])
+def test_prefill_head_dim_64(Hq, Hk, P, causal):
+    case = inputs.make_prefill_case(3, Hq, Hk, 64, P, [0, 70, 260], [33, 128, 150],
+                                    seed=Hq + Hk + P)
+    ref_o, ref_l = oracle_prefill(case, causal=causal)
+    out, lse = run_prefill(case, causal=causal)
+    check(out, lse, ref_o, ref_l, f"D=64 Hq={Hq} Hk={Hk} P={P} causal={causal}")
+
+
 def test_prefill_non_causal():
     case = inputs.make_prefill_case(2, 8, 2, 128, 16, [50, 200], [60, 129], seed=4)
     ref_o, ref_l = oracle_prefill(case, causal=False)
@@ -115,9 +125,18 @@ def test_chunked_prefill_full_config_sampled():
     assert np.isfinite(out).all()
 
 
-def _scaled_v_case(scale_v, seed):
+def test_chunked_prefill_full_config_every_row():
+    """The whole chunked-prefill workload (B=8, 512-token chunks after priors ~ U[0, 4096],
+    Hq=32, Hk=8, D=128, P=16), every output row against the oracle."""
+    case = inputs.chunked_prefill(seed=3)
+    out, lse = run_prefill(case)
+    ref_o, ref_l = oracle_prefill(case)
+    check(out, lse, ref_o, ref_l, "chunked prefill, every row")
+
+
+def _scaled_v_case(scale_v, seed, D=128):
     """The same chunked-prefill inputs with V multiplied by a power of two (exact in bf16)."""
-    case = inputs.make_prefill_case(3, 32, 8, 128, 16, [0, 300, 900], [77, 256, 160], seed=seed)
+    case = inputs.make_prefill_case(3, 32, 8, D, 16, [0, 300, 900], [77, 256, 160], seed=seed)
     kv = case.kv
     v = (kv.v_pages.float() * scale_v).to(torch.bfloat16)
     kv2 = inputs.PagedKV(kv.k_pages, v, kv.page_table, kv.seq_lens, kv.page_size)
@@ -135,3 +154,12 @@ def test_prefill_v_scale_covariance(log2s):
     ref_o, ref_l = oracle_prefill(base)
     out, lse = run_prefill(case)
     check(out / s, lse, ref_o, ref_l, f"V x 2^{log2s}")
+
+
+@pytest.mark.parametrize("log2s", [-12, 20])
+def test_prefill_v_scale_covariance_head_dim_64(log2s):
+    s = 2.0 ** log2s
+    base, case = _scaled_v_case(s, seed=31 + log2s, D=64)
+    ref_o, ref_l = oracle_prefill(base)
+    out, lse = run_prefill(case)
+    check(out / s, lse, ref_o, ref_l, f"D=64 V x 2^{log2s}")
