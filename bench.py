@@ -399,7 +399,7 @@ def parse(argv=None):
                     help="print one JSON document of a decode sweep instead of the bench line: "
                          "config3 = B x PackGQA x num_splits at ctx 2048 (bf16, e4m3); "
                          "splits = the split schedule's time per split count and (B, ctx)")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "long70b"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "long70b", "sparse70b"],
                     help="decode: the headline (paged GQA decode); prefill: causal chunked "
                          "prefill, B=8 chunks of 512 tokens after a prior context ~ U[0, 4096]; "
                          "long70b: B=4 decode at 8K/16K/24K/32K, Hq=64 Hk=8, page 64 (--kv)")
@@ -735,6 +735,134 @@ def measure_decode(a, dev, rank, world, dist, with_cpu):
     }
 
 
+# ------------------------------------------------------------------------ sparse decode
+
+SPARSE_TOPK, SPARSE_WINDOW = 32, 32
+SPARSE_METRIC = ("page-level top-K sparse GQA decode, 70B-shaped long context (B=4, ctx 8K-32K, "
+                 f"top {SPARSE_TOPK} pages of 64 + a {SPARSE_WINDOW}-token window): HBM GB/s of the "
+                 "bytes it reads (KT entries + chosen KV + q + out)")
+
+
+def sparse_step_bytes(sel_lens, seq_lens, Hq, Hk, D, P, topk, window):
+    """Algorithmic bytes of one sparse decode step: the KT entries of every scored page
+    (4*D bytes per (page, kv head); pages of the window are not scored, and nothing is
+    scored when the earlier pages are at most topk), the chosen tokens' K and V (bf16),
+    q and out."""
+    kt = 0
+    for L in seq_lens:
+        L = int(L)
+        np_ = (L + P - 1) // P
+        wp = min(max(L - window, 0) // P, np_) if window > 0 else np_
+        if wp > topk:
+            kt += wp * Hk * 4 * D
+    kv = 2 * sum(int(x) for x in sel_lens) * D * 2
+    B = len(seq_lens)
+    return kt + kv + 2 * B * Hq * D * 2, kt, kv
+
+
+def measure_sparse(a, dev, with_cpu):
+    import torch
+    from gqa_attention_paged_b200 import binding, inputs
+
+    case = inputs.long70b_decode(seed=a.seed, kv_dtype="bf16")
+    kv = case.kv
+    q, kp, vp = case.q.to(dev), kv.k_pages.to(dev), kv.v_pages.to(dev)
+    pt, sl = kv.page_table.to(dev), kv.seq_lens.to(dev)
+    B, Hq, D = case.q.shape
+    Hk, P = case.Hk, kv.page_size
+    topk, window = SPARSE_TOPK, SPARSE_WINDOW
+    kt = binding.gqa_paged_kt_build(kp, pt, sl)
+    ws = binding.new_workspace(binding.gqa_paged_sparse_decode_workspace_size(
+        B, Hq, Hk, D, P, pt.shape[1], topk, window, 0), dev)
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(on=None, qq=None, ptt=None, sll=None, oo=None, ll=None):
+        binding.gqa_paged_sparse_decode(q if qq is None else qq, kp, vp, kt,
+                                        pt if ptt is None else ptt, sl if sll is None else sll,
+                                        case.scale, topk, window, out=out if oo is None else oo,
+                                        lse=lse if ll is None else ll, workspace=ws,
+                                        stream=stream if on is None else on)
+
+    step()
+    torch.cuda.synchronize(dev)
+    assert binding.gqa_get_error(ws) == 0 and torch.isfinite(out.float()).all()
+    _, sel_lens, _ = binding.gqa_paged_sparse_select(q, kt, kp, pt, sl, topk, window)
+    torch.cuda.synchronize(dev)
+    step_bytes, kt_bytes, kv_bytes = sparse_step_bytes(sel_lens.tolist(), kv.seq_lens.tolist(),
+                                                       Hq, Hk, D, P, topk, window)
+    for _ in range(max(3, a.warmup)):
+        step()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    ms, sp = timed_graph(step, a.steps, stream, dev, a.repeat_seconds)
+    clk = clocks.stop()
+    # the dense decode of the same inputs, for the speedup
+    dws = binding.new_workspace(binding.gqa_paged_decode_workspace_size(
+        B, Hq, Hk, D, P, pt.shape[1] * P, 0, 0), dev)
+
+    def dense(on):
+        binding.gqa_paged_decode(q, kp, vp, pt, sl, case.scale, out=out, lse=lse, workspace=dws,
+                                 stream=on)
+
+    dense(stream)
+    dms, dsp = timed_graph(dense, a.steps, stream, dev, a.repeat_seconds)
+    hin = [case.q.pin_memory(), kv.page_table.pin_memory(), kv.seq_lens.pin_memory()]
+    din = [(q, q.clone()), (pt, pt.clone()), (sl, sl.clone())]
+    dout = [(out, torch.empty_like(out)), (lse, torch.empty_like(lse))]
+    hout = [(torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory()),
+            (torch.empty(B, Hq).pin_memory(), torch.empty(B, Hq).pin_memory())]
+
+    def run(s_, on):
+        step(on, din[0][s_], din[1][s_], din[2][s_], dout[0][s_], dout[1][s_])
+
+    e2e_ms = e2e_pipelined(dev, stream, hin, din, dout, hout, run, a.steps)
+    peak, kind = peaks()
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    cpu = None
+    if with_cpu:
+        from oracle import oracle
+        t0, reps = time.perf_counter(), 0
+        qb, kb, vb = _bits(case.q), _bits(kv.k_pages), _bits(kv.v_pages)
+        ptn, sln = kv.page_table.numpy(), kv.seq_lens.numpy()
+        while time.perf_counter() - t0 < min(a.cpu_seconds, 8.0):
+            ktn = oracle.kt_build(kb, ptn, sln) if reps == 0 else ktn
+            sc = oracle.page_scores(qb, ktn, ptn, sln, P)
+            sel, nsel = oracle.sparse_select(sc, sln, P, topk, window)
+            oracle.sparse_decode(qb, kb, vb, ptn, sln, case.scale, sel, nsel)
+            reps += 1
+        sec = (time.perf_counter() - t0) / reps
+        cpu = {"value": round(step_bytes / sec / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": f"the whole step (scores, selection, attention), {reps} "
+                                           "repeats (the first also builds the KT entries)"}
+    return {
+        "metric": SPARSE_METRIC, "value": round(gbs, 2), "unit": "GB/s",
+        "ms_per_step": round(ms, 5), "steps": a.steps, "warmup": max(3, a.warmup),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v, 1% outliers at 8 sigma)",
+        "config": {"workload": f"sparse decode B=4 ctx={{8K,16K,24K,32K}} Hq=64 Hk=8 D=128 P=64 "
+                               f"topk={topk} window={window}",
+                   "algorithmic_bytes_per_step": step_bytes, "kt_bytes": kt_bytes,
+                   "chosen_kv_bytes": kv_bytes, "chosen_tokens": int(sum(sel_lens.tolist())),
+                   "dense_tokens": int(Hk * kv.seq_lens.sum())},
+        "pct_of_hbm_peak": round(100 * gbs / peak, 2),
+        "dense_ms_per_step": round(dms, 5), "speedup_over_dense": round(dms / ms, 3),
+        "spread": sp,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "kernel": "sparse_select_kernel + decode_sk_kernel (+ piece merge): the whole call"},
+        "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hin),
+                "d2h_bytes_per_step": sum(p_[0].numel() * p_[0].element_size() for p_ in hout),
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": a.steps * (1 + binding.gqa_paged_decode_kernel_launches(
+            B * Hk, Hq // Hk, 1, D, P, binding.gqa_paged_sparse_table_stride(pt.shape[1], P, topk, window) * P,
+            0, 0)),
+        "clocks": clk, "cpu_baseline": cpu,
+    }
+
+
 # ------------------------------------------------------------------------ sweeps
 
 L2_BYTES = 126 << 20
@@ -832,26 +960,27 @@ def run_sweep(kind, a, dev):
                 del inp
                 torch.cuda.empty_cache()
     else:
-        grid = [(1, 512), (1, 2048), (1, 8192), (1, 32768), (4, 2048), (4, 8192), (4, 32768),
-                (16, 512), (16, 2048), (16, 8192), (16, 32768), (64, 512), (64, 2048),
-                (64, 8192), (256, 512), (256, 2048), (1024, 512), (1024, 1024)]
-        for B, ctx in grid:
-            inp = device_decode_inputs(B, ctx, Hq, Hk, D, P, "bf16", dev, seed=B + ctx)
-            for S in (1, 2, 4, 8, 16, 32):
-                if S > (ctx // P):
-                    continue
-                r = sweep_point(binding, inp, S, True, dev)
-                r.update({"B": B, "ctx": ctx, "num_splits": S})
-                res["points"].append(r)
-                print(json.dumps(r), file=sys.stderr, flush=True)
-            del inp
-            torch.cuda.empty_cache()
+        grid = [(B, ctx) for B in (1, 4, 16, 64, 256, 1024) for ctx in (512, 2048, 8192, 32768)
+                if B * ctx <= (2 << 20)]
+        for kv in ("bf16", "fp8_e4m3"):
+            for B, ctx in grid:
+                inp = device_decode_inputs(B, ctx, Hq, Hk, D, P, kv, dev, seed=B + ctx)
+                for S in (0, 1, 2, 4, 8, 16, 32, 64):
+                    if S > (ctx // P):
+                        continue
+                    r = sweep_point(binding, inp, S, True, dev)
+                    r.update({"B": B, "ctx": ctx, "kv": kv, "num_splits": "auto" if S == 0 else S})
+                    res["points"].append(r)
+                    print(json.dumps(r), file=sys.stderr, flush=True)
+                del inp
+                torch.cuda.empty_cache()
     return res
 
 
 def _secondary_summary(line):
     keep = ("metric", "value", "unit", "ms_per_step", "spread", "roofline", "clocks", "e2e",
-            "cpu_baseline", "gpu_launches", "pct_of_hbm_peak", "pct_of_bf16_peak", "dtype")
+            "cpu_baseline", "gpu_launches", "pct_of_hbm_peak", "pct_of_bf16_peak", "dtype",
+            "speedup_over_dense", "dense_ms_per_step")
     s = {k: line[k] for k in keep if k in line}
     s["workload"] = line["config"]["workload"]
     return s
@@ -880,10 +1009,11 @@ def main():
         if rank == 0:
             print(json.dumps(run_sweep(a.sweep, a, dev)))
         return 0
-    if a.workload == "prefill":
+    if a.workload in ("prefill", "sparse70b"):
         if rank != 0:
             return 0
-        line = measure_prefill(a, dev, with_cpu=not a.no_cpu_baseline)
+        fn = measure_prefill if a.workload == "prefill" else measure_sparse
+        line = fn(a, dev, with_cpu=not a.no_cpu_baseline)
         line.update({"n_gpus": 1, "scaling": "weak", "vs_baseline": None})
         print(json.dumps(line))
         return 0
@@ -910,6 +1040,9 @@ def main():
         la = parse(["--steps", str(a.steps), "--warmup", str(a.warmup), "--workload", "long70b",
                     "--kv", "fp8_e4m3", "--repeat-seconds", str(a.repeat_seconds)])
         sec.append(_secondary_summary(measure_decode(la, dev, 0, 1, None, with_cpu=False)))
+        sa = parse(["--steps", str(a.steps), "--warmup", str(a.warmup), "--workload", "sparse70b",
+                    "--repeat-seconds", str(a.repeat_seconds), "--cpu-seconds", str(a.cpu_seconds)])
+        sec.append(_secondary_summary(measure_sparse(sa, dev, with_cpu=not a.no_cpu_baseline)))
         line["secondary"] = sec
     print(json.dumps(line))
     return 0

@@ -39,8 +39,9 @@ SIGNATURES = {
     "gqa_paged_kt_build": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gqa_paged_kt_append": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gqa_paged_sparse_table_stride": (_I, [_I, _I, _I, _I]),
+    "gqa_paged_sparse_select_workspace_size": (_SZ, [_I, _I, _I]),
     "gqa_paged_sparse_select": (_I, [_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I,
-                                     _P, _P, _P, _P]),
+                                     _P, _P, _P, _SZ, _P]),
     "gqa_paged_sparse_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "gqa_paged_sparse_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                      ctypes.c_float, _I, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -531,11 +532,12 @@ def gqa_paged_sparse_select(q: torch.Tensor, kt: torch.Tensor, k_pages: torch.Te
     sel_pages = torch.full((B * Hk, max(ss, 1)), -1, dtype=torch.int32, device=dev)
     sel_lens = torch.zeros(B * Hk, dtype=torch.int32, device=dev)
     if workspace is None:
-        workspace = new_workspace(256, dev)
+        workspace = new_workspace(load().gqa_paged_sparse_select_workspace_size(B, Hk, pts), dev)
     st = load().gqa_paged_sparse_select(_ptr(q), _ptr(kt), _ptr(page_table), pts, _ptr(seq_lens),
                                         B, Hq, Hk, D, P, num_pages, int(topk), int(window),
                                         _ptr(sel_table), max(ss, 1), _ptr(sel_lens),
-                                        _ptr(sel_pages), _ptr(workspace), _stream(stream))
+                                        _ptr(sel_pages), _ptr(workspace), workspace.numel(),
+                                        _stream(stream))
     _check("gqa_paged_sparse_select", st)
     return sel_table, sel_lens, sel_pages
 

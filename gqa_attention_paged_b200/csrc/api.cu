@@ -495,11 +495,17 @@ int gqa_paged_sparse_table_stride(int pt_stride, int page_size, int topk, int wi
     return (int)(s < pt_stride ? s : pt_stride);
 }
 
+size_t gqa_paged_sparse_select_workspace_size(int B, int Hk, int pt_stride) {
+    if (B < 0 || Hk <= 0 || pt_stride <= 0) return 0;
+    return kWorkspaceHeader + align_up((size_t)B * Hk * pt_stride * sizeof(uint32_t), 256);
+}
+
 int gqa_paged_sparse_select(const void *q, const void *kt, const int32_t *page_table,
                             int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
                             int head_dim, int page_size, int num_pages, int topk, int window,
                             int32_t *sel_table, int sel_stride, int32_t *sel_lens,
-                            int32_t *sel_pages, void *workspace, cudaStream_t stream) {
+                            int32_t *sel_pages, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
     if (!q || !kt || !page_table || !seq_lens || !sel_table || !sel_lens || !workspace)
         return GQA_ERR_NULL;
     if (B < 0 || B > 65535 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 ||
@@ -510,13 +516,16 @@ int gqa_paged_sparse_select(const void *q, const void *kt, const int32_t *page_t
         (int64_t)num_pages * Hk * page_size > INT32_MAX)
         return GQA_ERR_SHAPE;
     if (!aligned(q, 16) || !aligned(kt, 16) || !aligned(page_table, 4) || !aligned(seq_lens, 4) ||
-        !aligned(sel_table, 4) || !aligned(sel_lens, 4) || (sel_pages && !aligned(sel_pages, 4)) ||
-        !aligned(workspace, 256))
+        !aligned(sel_table, 4) || !aligned(sel_lens, 4) || (sel_pages && !aligned(sel_pages, 4)))
         return GQA_ERR_ALIGN;
+    if (!aligned(workspace, 256) ||
+        workspace_bytes < gqa_paged_sparse_select_workspace_size(B, Hk, pt_stride))
+        return GQA_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
     return launch_sparse_select(q, kt, page_table, pt_stride, seq_lens, B, Hq, Hk, head_dim,
                                 page_size, num_pages, topk, window, sel_table, sel_stride,
-                                sel_lens, sel_pages, static_cast<int *>(workspace), stream) ==
-                   cudaSuccess
+                                sel_lens, sel_pages, reinterpret_cast<uint32_t *>(ws + kWorkspaceHeader),
+                                reinterpret_cast<int *>(ws), stream) == cudaSuccess
                ? GQA_OK
                : GQA_ERR_LAUNCH;
 }
@@ -531,7 +540,8 @@ size_t gqa_paged_sparse_decode_workspace_size(int B, int Hq, int Hk, int head_di
     return gqa_paged_decode_workspace_size(Bv, Hq / Hk, 1, head_dim, page_size, ss * page_size,
                                            GQA_KV_BF16, num_splits) +
            align_up((size_t)Bv * sizeof(int32_t), 256) +
-           align_up((size_t)Bv * ss * sizeof(int32_t), 256);
+           align_up((size_t)Bv * ss * sizeof(int32_t), 256) +
+           align_up((size_t)Bv * pt_stride * sizeof(uint32_t), 256);
 }
 
 int gqa_paged_sparse_decode(const void *q, const void *k_pages, const void *v_pages,
@@ -565,9 +575,11 @@ int gqa_paged_sparse_decode(const void *q, const void *k_pages, const void *v_pa
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int32_t *sel_lens = reinterpret_cast<int32_t *>(ws + dws);
     int32_t *sel_table = reinterpret_cast<int32_t *>(ws + dws + align_up((size_t)Bv * 4, 256));
+    uint32_t *keys = reinterpret_cast<uint32_t *>(ws + dws + align_up((size_t)Bv * 4, 256) +
+                                                  align_up((size_t)Bv * ss * 4, 256));
     if (launch_sparse_select(q, kt, page_table, pt_stride, seq_lens, B, Hq, Hk, head_dim,
                              page_size, num_pages, topk, window, sel_table, ss, sel_lens, nullptr,
-                             reinterpret_cast<int *>(ws), stream) != cudaSuccess)
+                             keys, reinterpret_cast<int *>(ws), stream) != cudaSuccess)
         return GQA_ERR_LAUNCH;
     // the chosen pages of every (sequence, kv head) as one sequence of a decode with one kv
     // head: q [B*Hk][g][D], pools [num_pages*Hk][1][P][D], out [B*Hk][g][D]

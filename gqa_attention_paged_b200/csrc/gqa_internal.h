@@ -141,12 +141,13 @@ cudaError_t launch_kt_build(const void *k_pages, const int32_t *page_table, int 
 cudaError_t launch_kt_append(const void *k_new, const int32_t *page_table, int pt_stride,
                              const int32_t *seq_lens, int B, int Hk, int D, int P, int num_pages,
                              void *kt, int *err, cudaStream_t stream);
-size_t sparse_select_smem_bytes(int g, int D, int pt_stride);
+// The scores of the selection go to `keys` [B*Hk][pt_stride] (order-preserving uint32).
 cudaError_t launch_sparse_select(const void *q, const void *kt, const int32_t *page_table,
                                  int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
                                  int D, int P, int num_pages, int topk, int window,
                                  int32_t *sel_table, int sel_stride, int32_t *sel_lens,
-                                 int32_t *sel_pages, int *err, cudaStream_t stream);
+                                 int32_t *sel_pages, uint32_t *keys, int *err,
+                                 cudaStream_t stream);
 // Largest page table (pages per sequence) and group the sparse selection takes.
 constexpr int kSparseMaxPages = 16384;
 constexpr int kSparseMaxGroup = 16;

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(256) kt_build_kernel(const uint16_t *__restric
         const uint32_t *src = reinterpret_cast<const uint32_t *>(
             k_pages + (((size_t)phys * Hk + kvh) * P) * D + d);
         float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
+#pragma unroll 8
         for (int t = 0; t < n; ++t) {
             const uint32_t w = __ldg(src + (size_t)t * (D / 2));
             const float v0 = bf16_bits_f32(w & 0xffffu), v1 = bf16_bits_f32(w >> 16);
@@ -150,30 +151,107 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int *red, int &total) 
     return r;
 }
 
-// One CTA per (kv head, sequence).  Shared memory: q of the group (fp32 [g][D]), one
-// round of KT rows (kSelChunk x (D + 1) words), the per-head partial scores, the scores
-// of all pages (as order-preserving keys after scoring), a 256-bin histogram and the
-// choice flags.
-__global__ void __launch_bounds__(kSelThreads) sparse_select_kernel(
+// First window page of a sequence of L tokens (np pages when the window is empty).
+__device__ __forceinline__ int window_first_page(int L, int np, int P, int window) {
+    const int lo = L - window > 0 ? L - window : 0;
+    return window > 0 ? min(lo / P, np) : np;
+}
+
+// Scores of the earlier (non-window) pages, kSelChunk pages per CTA: grid (page chunk,
+// kv head, sequence).  The chunk's page-table entries go to shared memory first, then its
+// KT rows (every load of a thread issued before the first store), padded to D + 1 words
+// per row so that the 32 lanes of a warp, each reading word d of its own page, hit 32
+// banks.  One thread per (page, query head) sums that head's D terms in order; one thread
+// per page then sums the heads in order.  The scores are written as order-preserving
+// keys to keys[(b * Hk + kvh) * pt_stride + page].
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) sparse_score_kernel(
     const uint16_t *__restrict__ q, const uint32_t *__restrict__ kt,
     const int32_t *__restrict__ page_table, int pt_stride, const int32_t *__restrict__ seq_lens,
-    int Hq, int Hk, int D, int P, int num_pages, int topk, int window,
+    int Hq, int Hk, int P, int num_pages, int topk, int window, uint32_t *__restrict__ keys,
+    int *err) {
+    constexpr int RW = D + 1;
+    constexpr int kWords = kSelChunk * D / kSelThreads;  // KT words each thread stages
+    __shared__ float qs[kSparseMaxGroup * D];
+    __shared__ uint32_t stage[kSelChunk * RW];
+    __shared__ float part[kSparseMaxGroup * kSelChunk];
+    __shared__ int phys_s[kSelChunk];
+    const int g = Hq / Hk;
+    const int kvh = blockIdx.y, b = blockIdx.z;
+    const int c0 = blockIdx.x * kSelChunk;
+    int L = seq_lens[b];
+    if (L < 0 || L > pt_stride * P) L = L < 0 ? 0 : pt_stride * P;  // reported by the pick kernel
+    const int np = (L + P - 1) / P;
+    const int wp = window_first_page(L, np, P, window);
+    if (wp <= topk || c0 >= wp) return;  // uniform for the CTA: nothing to score here
+    const int cn = min(kSelChunk, wp - c0);
+    for (int e = threadIdx.x; e < g * D; e += kSelThreads)
+        qs[e] = bf16_bits_f32(q[((size_t)b * Hq + kvh * g) * D + e]);
+    if (threadIdx.x < cn) {
+        int ph = page_table[(size_t)b * pt_stride + c0 + threadIdx.x];
+        if (ph < 0 || ph >= num_pages) {
+            set_error(err, GQA_ERR_BAD_PAGE);
+            ph = -1;  // scores as an all-zero box
+        }
+        phys_s[threadIdx.x] = ph;
+    }
+    __syncthreads();
+    uint32_t w[kWords];
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) {
+        const int e = threadIdx.x + k * kSelThreads;
+        const int i = e / D, d = e % D;
+        const int ph = i < cn ? phys_s[i] : -1;
+        w[k] = ph >= 0 ? __ldg(kt + ((size_t)ph * Hk + kvh) * D + d) : 0u;
+    }
+#pragma unroll
+    for (int k = 0; k < kWords; ++k) {
+        const int e = threadIdx.x + k * kSelThreads;
+        stage[(e / D) * RW + e % D] = w[k];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < g * kSelChunk; e += kSelThreads) {
+        const int i = e % kSelChunk, h = e / kSelChunk;
+        if (i >= cn) continue;
+        const float *qh = qs + h * D;
+        const uint32_t *r = stage + i * RW;
+        float sh = 0.f;
+#pragma unroll 8
+        for (int d = 0; d < D; ++d) {
+            const uint32_t x = r[d];
+            const float lo = qh[d] * bf16_bits_f32(x & 0xffffu);
+            const float hi = qh[d] * bf16_bits_f32(x >> 16);
+            sh = __fadd_rn(sh, lo > hi ? lo : hi);
+        }
+        part[h * kSelChunk + i] = sh;
+    }
+    __syncthreads();
+    if (threadIdx.x < cn) {
+        float tot = 0.f;
+        for (int h = 0; h < g; ++h) tot = __fadd_rn(tot, part[h * kSelChunk + threadIdx.x]);
+        keys[((size_t)b * Hk + kvh) * pt_stride + c0 + threadIdx.x] = score_key(tot);
+    }
+}
+
+// The choice per (kv head, sequence), one CTA each: the `topk` largest keys among the
+// earlier pages by radix select (8 bits a pass, most significant first; each pass a
+// histogram in shared memory and a warp scan over its 256 bins), the lowest pages first
+// among keys equal to the threshold, plus the window pages; then the chosen pages in
+// ascending order as physical * Hk + kvh, and their token count.
+__global__ void __launch_bounds__(kSelThreads) sparse_pick_kernel(
+    const uint32_t *__restrict__ keys_g, const int32_t *__restrict__ page_table, int pt_stride,
+    const int32_t *__restrict__ seq_lens, int Hk, int P, int num_pages, int topk, int window,
     int32_t *__restrict__ sel_table, int sel_stride, int32_t *__restrict__ sel_lens,
     int32_t *__restrict__ sel_pages, int *err) {
     extern __shared__ __align__(16) uint8_t smem[];
-    const int g = Hq / Hk;
-    const int kvh = blockIdx.x, b = blockIdx.y;
-    const int RW = D + 1;  // padded row: thread i reads word (i*RW + d), banks differ by i
-    float *qs = reinterpret_cast<float *>(smem);                 // [g][D]
-    uint32_t *stage = reinterpret_cast<uint32_t *>(qs + g * D);   // [kSelChunk][RW]
-    float *part = reinterpret_cast<float *>(stage + kSelChunk * RW);  // [g][kSelChunk]
-    uint32_t *keys = reinterpret_cast<uint32_t *>(part + g * kSelChunk);  // [pt_stride]
-    int *hist = reinterpret_cast<int *>(keys + pt_stride);        // [256]
-    int *red = hist + 256;                                        // [33]
-    uint8_t *take = reinterpret_cast<uint8_t *>(red + 40);        // [pt_stride]
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem);           // [pt_stride]
+    int *hist = reinterpret_cast<int *>(keys + pt_stride);         // [256]
+    int *red = hist + 256;                                         // [40]
+    uint8_t *take = reinterpret_cast<uint8_t *>(red + 40);         // [pt_stride]
     __shared__ uint32_t s_prefix;
     __shared__ int s_remaining;
-
+    const int kvh = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const size_t row = (size_t)b * Hk + kvh;
     int L = seq_lens[b];
     if (L < 0 || L > pt_stride * P) {
@@ -181,54 +259,12 @@ __global__ void __launch_bounds__(kSelThreads) sparse_select_kernel(
         L = L < 0 ? 0 : pt_stride * P;
     }
     const int np = (L + P - 1) / P;
-    const int lo_tok = L - window > 0 ? L - window : 0;
-    const int wp = window > 0 ? min(lo_tok / P, np) : np;  // first window page
+    const int wp = window_first_page(L, np, P, window);
     const int32_t *pt = page_table + (size_t)b * pt_stride;
     const bool dense = wp <= topk;
-
     for (int p = threadIdx.x; p < np; p += blockDim.x) take[p] = (dense || p >= wp) ? 1 : 0;
-
     if (!dense) {
-        // ---- scores of the earlier pages [0, wp)
-        for (int e = threadIdx.x; e < g * D; e += blockDim.x)
-            qs[e] = bf16_bits_f32(q[((size_t)b * Hq + kvh * g) * D + e]);
-        for (int c0 = 0; c0 < wp; c0 += kSelChunk) {
-            const int cn = min(kSelChunk, wp - c0);
-            __syncthreads();
-            for (int e = threadIdx.x; e < cn * D; e += blockDim.x) {
-                const int i = e / D, d = e % D;
-                const int phys = pt[c0 + i];
-                uint32_t w = 0u;  // a bad entry scores as an all-zero box
-                if (phys >= 0 && phys < num_pages)
-                    w = __ldg(kt + ((size_t)phys * Hk + kvh) * D + d);
-                else if (d == 0)
-                    set_error(err, GQA_ERR_BAD_PAGE);
-                stage[i * RW + d] = w;
-            }
-            __syncthreads();
-            for (int e = threadIdx.x; e < g * kSelChunk; e += blockDim.x) {
-                const int i = e % kSelChunk, h = e / kSelChunk;
-                if (i >= cn) continue;
-                const float *qh = qs + h * D;
-                const uint32_t *r = stage + i * RW;
-                float sh = 0.f;
-                for (int d = 0; d < D; ++d) {
-                    const uint32_t w = r[d];
-                    const float lo = qh[d] * bf16_bits_f32(w & 0xffffu);
-                    const float hi = qh[d] * bf16_bits_f32(w >> 16);
-                    sh = __fadd_rn(sh, lo > hi ? lo : hi);
-                }
-                part[h * kSelChunk + i] = sh;
-            }
-            __syncthreads();
-            for (int i = threadIdx.x; i < cn; i += blockDim.x) {
-                float tot = 0.f;
-                for (int h = 0; h < g; ++h) tot = __fadd_rn(tot, part[h * kSelChunk + i]);
-                keys[c0 + i] = score_key(tot);
-            }
-        }
-        // ---- the topk-th largest key T (radix select, 8 bits a pass, most significant
-        // first) and how many pages with key T to take (the lowest pages first)
+        for (int p = threadIdx.x; p < wp; p += blockDim.x) keys[p] = keys_g[row * pt_stride + p];
         if (threadIdx.x == 0) {
             s_prefix = 0u;
             s_remaining = topk;
@@ -243,14 +279,37 @@ __global__ void __launch_bounds__(kSelThreads) sparse_select_kernel(
                 if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 0xffu], 1);
             }
             __syncthreads();
-            if (threadIdx.x == 0) {
-                int rem = s_remaining, d = 255;
-                for (; d > 0; --d) {
-                    if (hist[d] >= rem) break;
-                    rem -= hist[d];
+            if (warp == 0) {
+                // lane l holds bins 255 - 8l ... 248 - 8l (descending); find the bin where the
+                // count from the top first reaches the remaining number
+                const int rem = s_remaining;
+                int cnt[8], sum = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    cnt[k] = hist[255 - 8 * lane - k];
+                    sum += cnt[k];
                 }
-                s_prefix = prefix | ((uint32_t)d << shift);
-                s_remaining = rem;
+                int incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);
+                const int lw = hit ? __ffs(hit) - 1 : 31;
+                if (lane == lw) {
+                    int r = rem - (incl - sum), d = 255 - 8 * lane;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        if (cnt[k] >= r || k == 7) {
+                            d = 255 - 8 * lane - k;
+                            break;
+                        }
+                        r -= cnt[k];
+                    }
+                    s_prefix = prefix | ((uint32_t)d << shift);
+                    s_remaining = r;
+                }
             }
             mask |= 0xffu << shift;
             __syncthreads();
@@ -324,25 +383,35 @@ cudaError_t launch_kt_append(const void *k_new, const int32_t *page_table, int p
     return cudaGetLastError();
 }
 
-size_t sparse_select_smem_bytes(int g, int D, int pt_stride) {
-    return sizeof(float) * ((size_t)g * D + (size_t)kSelChunk * (D + 1) + (size_t)g * kSelChunk) +
-           sizeof(uint32_t) * (size_t)pt_stride + sizeof(int) * (256 + 40) + (size_t)pt_stride + 16;
+size_t sparse_pick_smem_bytes(int pt_stride) {
+    return sizeof(uint32_t) * (size_t)pt_stride + sizeof(int) * (256 + 40) + (size_t)pt_stride + 16;
 }
 
 cudaError_t launch_sparse_select(const void *q, const void *kt, const int32_t *page_table,
                                  int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
                                  int D, int P, int num_pages, int topk, int window,
                                  int32_t *sel_table, int sel_stride, int32_t *sel_lens,
-                                 int32_t *sel_pages, int *err, cudaStream_t stream) {
+                                 int32_t *sel_pages, uint32_t *keys, int *err,
+                                 cudaStream_t stream) {
     if (B == 0) return cudaSuccess;
-    const size_t smem = sparse_select_smem_bytes(Hq / Hk, D, pt_stride);
-    cudaError_t e = cudaFuncSetAttribute(sparse_select_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const dim3 sgrid((pt_stride + kSelChunk - 1) / kSelChunk, Hk, B);
+    if (D == 128)
+        sparse_score_kernel<128><<<sgrid, kSelThreads, 0, stream>>>(
+            static_cast<const uint16_t *>(q), static_cast<const uint32_t *>(kt), page_table,
+            pt_stride, seq_lens, Hq, Hk, P, num_pages, topk, window, keys, err);
+    else
+        sparse_score_kernel<64><<<sgrid, kSelThreads, 0, stream>>>(
+            static_cast<const uint16_t *>(q), static_cast<const uint32_t *>(kt), page_table,
+            pt_stride, seq_lens, Hq, Hk, P, num_pages, topk, window, keys, err);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    sparse_select_kernel<<<dim3(Hk, B), kSelThreads, smem, stream>>>(
-        static_cast<const uint16_t *>(q), static_cast<const uint32_t *>(kt), page_table,
-        pt_stride, seq_lens, Hq, Hk, D, P, num_pages, topk, window, sel_table, sel_stride,
-        sel_lens, sel_pages, err);
+    const size_t smem = sparse_pick_smem_bytes(pt_stride);
+    e = cudaFuncSetAttribute(sparse_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    sparse_pick_kernel<<<dim3(Hk, B), kSelThreads, smem, stream>>>(
+        keys, page_table, pt_stride, seq_lens, Hk, P, num_pages, topk, window, sel_table,
+        sel_stride, sel_lens, sel_pages, err);
     return cudaGetLastError();
 }
 

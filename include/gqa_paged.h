@@ -381,6 +381,10 @@ int gqa_paged_kt_append(const void *k_new, const int32_t *page_table, int pt_str
  */
 int gqa_paged_sparse_table_stride(int pt_stride, int page_size, int topk, int window);
 
+/* Workspace of gqa_paged_sparse_select(): the error-word header, then the page scores
+ * (one 32-bit key per (sequence, kv head, page)). */
+size_t gqa_paged_sparse_select_workspace_size(int B, int Hk, int pt_stride);
+
 /*
  * The selection alone.  For row r = b * Hk + j (sequence b, kv head j):
  *   sel_table int32 [B*Hk][sel_stride]: the chosen pages in ascending logical order, each
@@ -389,16 +393,19 @@ int gqa_paged_sparse_table_stride(int pt_stride, int page_size, int topk, int wi
  *   sel_lens  int32 [B*Hk]: tokens in the chosen pages
  *   sel_pages int32 [B*Hk][sel_stride] or NULL: the chosen logical page indices
  *   sel_stride >= gqa_paged_sparse_table_stride(pt_stride, page_size, topk, window)
- * workspace: >= 256 bytes, 256-byte aligned (error word).
+ * workspace: >= gqa_paged_sparse_select_workspace_size(B, Hk, pt_stride) bytes, 256-byte
+ * aligned, zeroed before first use (error word, then the scores between the two kernels:
+ * one scores pages in chunks of 64 over a (chunk, kv head, sequence) grid, one picks).
  */
 int gqa_paged_sparse_select(const void *q, const void *kt, const int32_t *page_table,
                             int pt_stride, const int32_t *seq_lens, int B, int Hq, int Hk,
                             int head_dim, int page_size, int num_pages, int topk, int window,
                             int32_t *sel_table, int sel_stride, int32_t *sel_lens,
-                            int32_t *sel_pages, void *workspace, cudaStream_t stream);
+                            int32_t *sel_pages, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
 
 /* Workspace of gqa_paged_sparse_decode(): the decode's for B*Hk sequences of one kv head
- * and g = Hq/Hk heads, then the chosen-page lengths and table. */
+ * and g = Hq/Hk heads, then the chosen-page lengths and table, then the page scores. */
 size_t gqa_paged_sparse_decode_workspace_size(int B, int Hq, int Hk, int head_dim,
                                               int page_size, int pt_stride, int topk, int window,
                                               int num_splits);

@@ -92,7 +92,9 @@ def _check_selection(case, d, topk, window, pt=None):
     pt_h = kv.page_table if pt is None else pt
     pt_d = pt_h.to(DEV)
     kt = binding.gqa_paged_kt_build(d["k"], pt_d, d["sl"])
-    ws = binding.new_workspace(256, DEV)
+    B, Hk = kv.page_table.shape[0], kv.k_pages.shape[1]
+    ws = binding.new_workspace(binding.load().gqa_paged_sparse_select_workspace_size(
+        B, Hk, pt_h.shape[1]), DEV)
     st, sl_, sp = binding.gqa_paged_sparse_select(d["q"], kt, d["k"], pt_d, d["sl"], topk, window,
                                                   workspace=ws)
     assert binding.gqa_get_error(ws) == 0
