@@ -965,11 +965,12 @@ def run_sweep(kind, a, dev):
         for kv in ("bf16", "fp8_e4m3"):
             for B, ctx in grid:
                 inp = device_decode_inputs(B, ctx, Hq, Hk, D, P, kv, dev, seed=B + ctx)
-                for S in (0, 1, 2, 4, 8, 16, 32, 64):
+                for S in (-1, 0, 1, 2, 4, 8, 16, 32, 64):
                     if S > (ctx // P):
                         continue
                     r = sweep_point(binding, inp, S, True, dev)
-                    r.update({"B": B, "ctx": ctx, "kv": kv, "num_splits": "auto" if S == 0 else S})
+                    r.update({"B": B, "ctx": ctx, "kv": kv,
+                              "num_splits": {-1: "balanced", 0: "auto"}.get(S, S)})
                     res["points"].append(r)
                     print(json.dumps(r), file=sys.stderr, flush=True)
                 del inp

@@ -22,6 +22,7 @@ GQA_OK = 0
 GQA_KV_BF16 = 0
 GQA_KV_FP8_E4M3 = 1
 GQA_MAX_SPLITS = 64
+GQA_SPLITS_BALANCED = -1
 
 _lib = None
 _P = ctypes.c_void_p

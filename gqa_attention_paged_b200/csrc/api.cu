@@ -3,6 +3,7 @@
 // memory is allocated here; every buffer is the caller's.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -72,12 +73,54 @@ int encode_q_map(CUtensorMap *map, const void *q, int total_q, int Hq, int D, in
 
 bool valid_page_size(int P) { return P == 16 || P == 32 || P == 64; }
 
-int resolve_splits(int num_splits, int B, int Hk, int pt_stride, int P, int kv_dtype) {
-    if (num_splits > 0) return num_splits;
-    return gqa_pick_splits(B, Hk, pt_stride * P, P, kv_dtype);
+int sm_count();
+
+// Split counts measured on one B200 (148 SMs) with `bench.py --sweep splits` (decode_sweep
+// under profiles/): Hq=32, Hk=8, head_dim 128, page 16, every sequence the same length;
+// rows: units B*Hk of 8, 32, 128, 512, 2048, 8192; columns: context 512, 2048, 8192,
+// 32768 tokens; [0] bf16 KV, [1] e4m3 KV.  Cells with B * context above 2M tokens were not
+// measured and repeat their measured neighbour.
+//   kBestSplits: the split schedule's fastest split count (gqa_pick_splits).
+//   kAutoSplits: what num_splits = 0 runs: 0 = the balanced schedule, else that split
+//     count, where the split schedule measured at least 5% faster than the balanced one
+//     (a few short sequences).
+constexpr int kTabUnits = 6, kTabCtx = 4;
+const unsigned char kBestSplits[2][kTabUnits][kTabCtx] = {
+    {{8, 16, 32, 32}, {4, 8, 8, 32}, {2, 2, 16, 16}, {2, 4, 4, 16}, {1, 1, 4, 4}, {1, 1, 1, 1}},
+    {{8, 16, 32, 32}, {4, 8, 8, 32}, {2, 2, 16, 16}, {1, 4, 4, 16}, {1, 1, 4, 4}, {1, 1, 1, 1}}};
+const unsigned char kAutoSplits[2][kTabUnits][kTabCtx] = {
+    {{8, 0, 0, 0}, {4, 8, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}},
+    {{8, 16, 0, 0}, {4, 8, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}}};
+
+// Table cell of (units, context): the nearest row and column in log scale (rows and
+// columns are a factor 4 apart); units are first scaled to 148 SMs.
+void split_cell(int B, int Hk, int max_seq_len, int &ui, int &ci) {
+    double units = (double)B * Hk * 148.0 / (double)sm_count();
+    double ctx = max_seq_len > 0 ? (double)max_seq_len : 1.0;
+    int u = (int)lround(log(units / 8.0) / log(4.0));
+    int c = (int)lround(log(ctx / 512.0) / log(4.0));
+    ui = u < 0 ? 0 : (u >= kTabUnits ? kTabUnits - 1 : u);
+    ci = c < 0 ? 0 : (c >= kTabCtx ? kTabCtx - 1 : c);
 }
 
-bool use_stream_k(int num_splits, int B) { return num_splits == 0 && B <= kStreamMaxBatch; }
+int clamp_splits(int s, int max_seq_len, int P) {
+    const int pages = (max_seq_len + P - 1) / P;
+    if (s > pages) s = pages;
+    if (s > GQA_MAX_SPLITS) s = GQA_MAX_SPLITS;
+    return s < 1 ? 1 : s;
+}
+
+// The schedule a decode call runs: 0 = balanced persistent, else the split schedule with
+// that many splits.
+int decode_schedule(int num_splits, int B, int Hk, int max_seq_len, int P, int kv_dtype) {
+    if (num_splits > 0) return num_splits;
+    if (B > kStreamMaxBatch) return gqa_pick_splits(B, Hk, max_seq_len, P, kv_dtype);
+    if (num_splits == GQA_SPLITS_BALANCED || B <= 0 || Hk <= 0 || P <= 0) return 0;
+    int ui, ci;
+    split_cell(B, Hk, max_seq_len, ui, ci);
+    const int s = kAutoSplits[kv_dtype == GQA_KV_FP8_E4M3 ? 1 : 0][ui][ci];
+    return s == 0 ? 0 : clamp_splits(s, max_seq_len, P);
+}
 
 // Merge-piece slots of the balanced schedule: 2 per worker, for the largest grid.
 size_t stream_k_piece_bytes(int Hq, int Hk, int D) {
@@ -88,7 +131,6 @@ size_t stream_k_piece_bytes(int Hq, int Hk, int D) {
     return align_up(slots * slot_floats * sizeof(float), 256);
 }
 
-int sm_count();
 
 // CTAs of the balanced decode schedule: kStreamCtasPerSm per SM.
 int decode_grid() {
@@ -128,7 +170,7 @@ int decode_check_args(const void *q, const void *k_pages, const void *v_pages,
         pt_stride <= 0 || (int64_t)num_pages * Hk * page_size > INT32_MAX ||
         (int64_t)pt_stride * page_size > INT32_MAX)
         return GQA_ERR_SHAPE;
-    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (num_splits < GQA_SPLITS_BALANCED || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
     if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
         !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
         return GQA_ERR_ALIGN;
@@ -146,11 +188,12 @@ int decode_call(const void *q, const void *k_pages, const void *v_pages, const f
                                       num_pages, num_splits, out, lse);
     if (chk != GQA_OK) return chk;
     if (!workspace) return GQA_ERR_NULL;
-    const bool sk = use_stream_k(num_splits, B);
-    const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
+    const int sched = decode_schedule(num_splits, B, Hk, pt_stride * page_size, page_size, kv_dtype);
+    const bool sk = sched == 0;
+    const int S = sk ? 1 : sched;
     const size_t need = gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
                                                         pt_stride * page_size, kv_dtype,
-                                                        sk ? 0 : S);
+                                                        num_splits);
     if (!aligned(workspace, 256) || workspace_bytes < need) return GQA_ERR_WORKSPACE;
     if (B == 0) return GQA_OK;
 
@@ -221,27 +264,18 @@ const char *gqa_status_string(int s) {
 }
 
 int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype) {
-    (void)kv_dtype;
-    if (B <= 0 || Hk <= 0 || page_size <= 0) return 1;
-    const int pages = (max_seq_len + page_size - 1) / page_size;
-    const int tiles = (max_seq_len + 15) / 16;
-    const int units = B * Hk;
-    const int slots = 148 * 3;  // SMs x resident decode CTAs per SM
-    // enough CTAs for ~4 waves, but keep >= 16 tiles of work per split
-    int s = (4 * slots + units - 1) / units;
-    const int max_by_work = tiles / 16 > 0 ? tiles / 16 : 1;
-    if (s > max_by_work) s = max_by_work;
-    if (s > pages) s = pages > 0 ? pages : 1;
-    if (s > GQA_MAX_SPLITS) s = GQA_MAX_SPLITS;
-    return s < 1 ? 1 : s;
+    if (B <= 0 || Hk <= 0 || page_size <= 0 || max_seq_len <= 0) return 1;
+    int ui, ci;
+    split_cell(B, Hk, max_seq_len, ui, ci);
+    return clamp_splits(kBestSplits[kv_dtype == GQA_KV_FP8_E4M3 ? 1 : 0][ui][ci], max_seq_len,
+                        page_size);
 }
 
 size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int page_size,
                                        int max_seq_len, int kv_dtype, int num_splits) {
-    if (use_stream_k(num_splits, B) && Hq > 0 && Hk > 0 && Hq % Hk == 0)
+    const int S = decode_schedule(num_splits, B, Hk, max_seq_len, page_size, kv_dtype);
+    if (S == 0 && Hq > 0 && Hk > 0 && Hq % Hk == 0)
         return decode_zero_prefix_bytes(B, Hq) + stream_k_piece_bytes(Hq, Hk, head_dim);
-    int S = num_splits > 0 ? num_splits
-                           : gqa_pick_splits(B, Hk, max_seq_len, page_size, kv_dtype);
     size_t bytes = kWorkspaceHeader;
     if (S > 1) {
         const size_t rows = (size_t)B * Hq;
@@ -256,10 +290,8 @@ int gqa_paged_decode_kernel_launches(int B, int Hq, int Hk, int head_dim, int pa
                                      int pack_gqa) {
     (void)head_dim;
     if (B <= 0 || Hq <= 0 || Hk <= 0 || Hq % Hk != 0 || page_size <= 0) return 0;
-    if (use_stream_k(num_splits, B))
-        return decode_defers_merge(B, Hq, Hk, pack_gqa ? 1 : 0, decode_grid()) ? 2 : 1;
-    const int S = num_splits > 0 ? num_splits
-                                 : gqa_pick_splits(B, Hk, max_seq_len, page_size, kv_dtype);
+    const int S = decode_schedule(num_splits, B, Hk, max_seq_len, page_size, kv_dtype);
+    if (S == 0) return decode_defers_merge(B, Hq, Hk, pack_gqa ? 1 : 0, decode_grid()) ? 2 : 1;
     return S > 1 ? 2 : 1;
 }
 
@@ -431,17 +463,15 @@ int gqa_paged_append_decode(const void *q, const void *k_new, const void *v_new,
     // the decode's checks first, so that a call it would reject changes nothing
     if (!q || !out) return GQA_ERR_NULL;
     if (Hq <= 0 || Hk <= 0 || Hq % Hk != 0) return GQA_ERR_SHAPE;
-    if (num_splits < 0 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (num_splits < GQA_SPLITS_BALANCED || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
     if (kv_dtype == GQA_KV_FP8_E4M3 && head_dim != 128) return GQA_ERR_DTYPE;
     if (!workspace || !aligned(workspace, 256)) return workspace ? GQA_ERR_WORKSPACE : GQA_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
         (lse && !aligned(lse, 4)))
         return GQA_ERR_ALIGN;
-    const bool sk = use_stream_k(num_splits, B);
-    const int S = sk ? 1 : resolve_splits(num_splits, B, Hk, pt_stride, page_size, kv_dtype);
     if (workspace_bytes < gqa_paged_decode_workspace_size(B, Hq, Hk, head_dim, page_size,
                                                           pt_stride * page_size, kv_dtype,
-                                                          sk ? 0 : S))
+                                                          num_splits))
         return GQA_ERR_WORKSPACE;
     const int r = gqa_paged_append_kv(k_new, v_new, k_pages, v_pages, k_scale, v_scale,
                                       kv_dtype, page_table, pt_stride, seq_lens, B, Hk,

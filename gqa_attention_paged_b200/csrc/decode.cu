@@ -127,12 +127,8 @@ struct WarpAttn {
     float o[NT][KT][4];
     float m[NT][2], l[NT][2];  // reference (log2 units) and running sum per head column
 
-    __device__ __forceinline__ static int dim0(int dt, int gq) {
-        return FP8 ? dt * 16 + 4 * (gq >> 1) + (gq & 1) : dt * 16 + gq;
-    }
-    __device__ __forceinline__ static int dim1(int dt, int gq) {
-        return FP8 ? dim0(dt, gq) + 2 : dim0(dt, gq) + 8;
-    }
+    __device__ __forceinline__ static int dim0(int dt, int gq) { return dt * 16 + gq; }
+    __device__ __forceinline__ static int dim1(int dt, int gq) { return dt * 16 + gq + 8; }
 
     __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -239,6 +235,13 @@ struct WarpAttn {
                 }
             }
         } else {
+            // the even and odd k steps accumulate in two chains, added at the end: half the
+            // dependent MMA latency per 16-token half
+            float s2[MT][NT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) s2[mt][nt][0] = s2[mt][nt][1] = s2[mt][nt][2] = s2[mt][nt][3] = 0.f;
             // One ldmatrix.x4 over 32 fp8 dims serves two k steps; the k order inside a
             // step is permuted identically for K (here) and q (qf), which leaves each dot
             // product unchanged.
@@ -250,17 +253,24 @@ struct WarpAttn {
                 for (int kp = 0; kp < D / 32; ++kp) {
                     uint32_t raw[4];
                     ldsm_x4(raw, kbase + swz<TT>(r, 32 * kp + (j >> 1) * 16));
-                    uint32_t a0[4] = {e4m3x2_to_f16x2(raw[0] & 0xffff), e4m3x2_to_f16x2(raw[1] & 0xffff),
-                                      e4m3x2_to_f16x2(raw[0] >> 16), e4m3x2_to_f16x2(raw[1] >> 16)};
-                    uint32_t a1[4] = {e4m3x2_to_f16x2(raw[2] & 0xffff), e4m3x2_to_f16x2(raw[3] & 0xffff),
-                                      e4m3x2_to_f16x2(raw[2] >> 16), e4m3x2_to_f16x2(raw[3] >> 16)};
+                    uint32_t a0[4], a1[4];
+                    e4m3x4_to_f16x4(raw[0], a0[0], a0[2]);
+                    e4m3x4_to_f16x4(raw[1], a0[1], a0[3]);
+                    e4m3x4_to_f16x4(raw[2], a1[0], a1[2]);
+                    e4m3x4_to_f16x4(raw[3], a1[1], a1[3]);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
                         mma_f16(s[mt][nt], a0, qf[nt][2 * kp][0], qf[nt][2 * kp][1]);
-                        mma_f16(s[mt][nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
+                        mma_f16(s2[mt][nt], a1, qf[nt][2 * kp + 1][0], qf[nt][2 * kp + 1][1]);
                     }
                 }
             }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[mt][nt][e] += s2[mt][nt][e];
         }
 
         // ---- online softmax (exp2 domain) over the tile, per packed head column, with a
@@ -378,27 +388,26 @@ struct WarpAttn {
                 }
             }
         } else {
-            // fp8 V: plain ldmatrix gives each lane 4 consecutive dims of one token;
-            // after conversion, movmatrix transposes 8x8 blocks into the A layout (dims
-            // permuted within each 16-dim tile; dim0/dim1 undo it when O is written).
-            const int j = lane >> 3;
+            // fp8 V: a transposing byte ldmatrix per 16 tokens x 16 dims gives each lane
+            // four tokens of one dim, already in the A fragment's k order once the rows are
+            // fed permuted: matrix row i (lane i < 16 gives its address) is token pi(i) of
+            // the 16-token half, pi(4c + k) = 2c + (k & 1) + 8 (k >> 1), so lane (g, c)
+            // receives tokens 2c, 2c+1, 2c+8, 2c+9 of dims g and g+8; two conversions make
+            // the four f16 pairs, with no transpose through registers.
+            const int ii = lane & 15;
+            const int tok = 2 * (ii >> 2) + (ii & 1) + 8 * ((ii >> 1) & 1);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const int r = (lane & 7) + (j & 1) * 8 + 16 * mt;
+                const int r = tok + 16 * mt;
 #pragma unroll
-                for (int qd = 0; qd < D / 32; ++qd) {
-                    uint32_t raw[4];
-                    ldsm_x4(raw, vbase + swz<TT>(r, 32 * qd + (j >> 1) * 16));
+                for (int dt = 0; dt < KT; ++dt) {
+                    uint32_t w0, w1;
+                    ldsm8_trans_x1(w0, w1, vbase + swz<TT>(r, 16 * dt));
+                    uint32_t af[4];
+                    e4m3x4_to_f16x4(w0, af[0], af[2]);
+                    e4m3x4_to_f16x4(w1, af[1], af[3]);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t lo_t = raw[2 * h], hi_t = raw[2 * h + 1];  // tokens 0-7 / 8-15
-                        uint32_t af[4] = {movmatrix_trans(e4m3x2_to_f16x2(lo_t & 0xffff)),
-                                          movmatrix_trans(e4m3x2_to_f16x2(lo_t >> 16)),
-                                          movmatrix_trans(e4m3x2_to_f16x2(hi_t & 0xffff)),
-                                          movmatrix_trans(e4m3x2_to_f16x2(hi_t >> 16))};
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) mma_f16(o[nt][2 * qd + h], af, pb[mt][nt][0], pb[mt][nt][1]);
-                    }
+                    for (int nt = 0; nt < NT; ++nt) mma_f16(o[nt][dt], af, pb[mt][nt][0], pb[mt][nt][1]);
                 }
             }
         }
@@ -640,16 +649,18 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 // producer lane (lane w of warp 4), so a warp that pauses (loading the next unit's q,
 // merging pieces) never holds up the other warps' streams.
 
-constexpr int kMinTilesPerWorker = 16;
+constexpr int kMinTilesPerWorker = 16;  // 16-token tiles; half as many 32-token tiles
 // When one worker per kMinTilesPerWorker tiles would leave more than three quarters of the
 // workers idle (a few short sequences), one per kMinTilesPerWorkerSmall tiles: such
 // streams are latency-bound, so more of them in flight finish sooner.
 constexpr int kMinTilesPerWorkerSmall = 4;
 
-// Workers of a launch with T tiles and `workers` consumer warps.
+// Workers of a launch with T tiles of TT tokens and `workers` consumer warps.
+template <int TT>
 __device__ __forceinline__ long long sk_workers(long long T, long long workers) {
-    const long long nw = T / kMinTilesPerWorker;
-    const long long per = nw * 4 < workers ? kMinTilesPerWorkerSmall : kMinTilesPerWorker;
+    constexpr long long kMin = kMinTilesPerWorker * 16 / TT;
+    const long long nw = T / kMin;
+    const long long per = nw * 4 < workers ? kMinTilesPerWorkerSmall : kMin;
     return min(workers, max(1LL, T / per));
 }
 // Launches whose units average more than kDeferMinWorkersPerUnit workers each leave their
@@ -830,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm)
     __syncthreads();
 
     const long long T = (long long)U * pre[B];
-    const long long NW = sk_workers(T, (long long)gridDim.x * kConsumerWarps);
+    const long long NW = sk_workers<TT>(T, (long long)gridDim.x * kConsumerWarps);
     const long long W0cta = (long long)blockIdx.x * kConsumerWarps;
 
     // Sequences with no tokens have no tiles: their outputs are written here (zeros, -inf).
@@ -1073,7 +1084,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
     if (warp == 0) tile_prefix<TT>(a, pre_m, a.pt_stride * a.P, nullptr, lane);
     __syncthreads();
     const long long T = (long long)U * pre_m[a.B];
-    const long long NW = sk_workers(T, (long long)a.grid * kConsumerWarps);
+    const long long NW = sk_workers<TT>(T, (long long)a.grid * kConsumerWarps);
     const int slot_floats = (heads_per_cta * (D + 1) + 3) & ~3;
     for (long long u = blockIdx.x; u < (long long)a.B * U; u += gridDim.x) {
         const int b = (int)(u / U), y = (int)(u % U);

@@ -149,6 +149,15 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
                  : "r"(addr));
 }
 
+// A 16 x 16 matrix of bytes, transposed: lanes 0-15 give the addresses of its 16 rows
+// (16 bytes each); lane l receives rows 4(l % 4) .. 4(l % 4) + 3 of column l / 4 in r0 (row
+// 4(l % 4) in the low byte) and the same rows of column l / 4 + 8 in r1 (lane layout
+// checked on a B200 with a matrix of known bytes).
+__device__ __forceinline__ void ldsm8_trans_x1(uint32_t &r0, uint32_t &r1, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x1.trans.shared.b8 {%0,%1}, [%2];"
+                 : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -223,13 +232,16 @@ __device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsig
     return d;
 }
 
-// Two e4m3 bytes (low byte first) -> f16x2 (exact: every e4m3 value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-}
-
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+
+// Four e4m3 bytes (byte 0 lowest) -> two f16x2 words: lo from bytes 0-1, hi from 2-3
+// (exact: every e4m3 value is an f16 value).  The 32-bit word is split into its 16-bit
+// halves in PTX, so each half feeds one conversion directly.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi) : "r"(w));
+}
 
 // ----------------------------------------------------------------------------------------
 // Tensor memory (TMEM) and 5th-generation tensor-core MMA (tcgen05), single-CTA form.

@@ -73,6 +73,9 @@ typedef enum {
 } gqa_kv_dtype_t;
 
 #define GQA_MAX_SPLITS 64
+/* num_splits value that asks for the balanced persistent schedule whatever the problem
+ * size (B <= 2048), for comparison sweeps; 0 lets the measured table decide. */
+#define GQA_SPLITS_BALANCED (-1)
 
 /*
  * Bytes of workspace gqa_paged_decode() needs for the same B, heads, head_dim, page_size,
@@ -98,9 +101,11 @@ int gqa_paged_decode_kernel_launches(int B, int Hq, int Hk, int head_dim, int pa
                                      int pack_gqa);
 
 /*
- * Split count gqa_paged_decode() uses with num_splits = 0 when B is above the balanced
- * schedule's limit (2048): chosen from B, kv heads Hk and the longest context (tokens)
- * to give several waves of CTAs with at least 16 tiles of work each.
+ * The split schedule's measured fastest split count for B sequences of Hk kv heads and
+ * context max_seq_len: a table measured on one B200 over units (B * Hk, scaled to this
+ * device's SM count) and context, for bf16 and e4m3 KV, nearest entry in log scale.
+ * gqa_paged_decode() uses it with num_splits = 0 when B is above the balanced schedule's
+ * limit (2048).
  */
 int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype);
 
@@ -123,8 +128,11 @@ int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype)
  *   num_splits 0 = automatic: for B <= 2048 a balanced persistent schedule: all
  *              (sequence, kv head) tiles of 16 tokens are laid end to end and shared
  *              equally by the workers of a fixed grid, and units cut between workers are
- *              merged by log-sum-exp inside the same launch; for larger B, splits as
- *              below with the count gqa_pick_splits gives for context pt_stride*page_size.
+ *              merged by log-sum-exp inside the same launch -- except for the small
+ *              problems (a few sequences of short context pt_stride*page_size) where the
+ *              split schedule measured faster, which run splits with the measured count;
+ *              for larger B, splits with the count gqa_pick_splits gives.
+ *              GQA_SPLITS_BALANCED (-1): the balanced schedule for any B <= 2048.
  *              1..GQA_MAX_SPLITS: contiguous page-aligned ranges of ceil(np / num_splits)
  *              pages (np = ceil(seq_len / page_size)), merged with lse_combine on the
  *              same stream

@@ -77,7 +77,7 @@ def _decode(**kw):
     (dict(Hq=6, Hk=4), -2), (dict(D=96), -2), (dict(P=8), -2), (dict(P=128), -2),
     (dict(npg=0), -2), (dict(pts=0), -2), (dict(B=-1), -2), (dict(B=70000), -2),
     (dict(kvd=5), -3), (dict(kvd=1), -3), (dict(kvd=1, ks=_fake(), vs=_fake(), D=64), -3),
-    (dict(S=-1), -4), (dict(S=65), -4),
+    (dict(S=-2), -4), (dict(S=65), -4),
     (dict(q=_fake(0x10008)), -9), (dict(k=_fake(0x10004)), -9),
     (dict(ws=_fake(0x10010)), -5), (dict(wsb=16), -5),
     (dict(S=4, wsb=256), -5),
@@ -170,7 +170,7 @@ def _static(**kw):
     # then the size check: 64 splits of B=64 need more than the fixed array
     (dict(B=64, S=64), -5),
     # groups of more than 8 heads at head_dim 128 never fit the balanced schedule's pieces
-    (dict(Hq=128, Hk=8, S=0), -5), (dict(Hq=16, Hk=1, S=0), -5),
+    (dict(Hq=128, Hk=8, S=0), -5), (dict(B=256, Hq=16, Hk=1, S=0), -5),
 ])
 def test_static_scratch_rejects_on_the_host(kw, status):
     """These pointers are never dereferenced: every rejection happens on the host."""
@@ -181,3 +181,27 @@ def test_static_scratch_fits_groups_above_8_with_splits():
     lib = binding.load()
     assert lib.gqa_paged_decode_workspace_size(16, 128, 8, 128, 16, 2048, 0, 0) > 16 << 20
     assert lib.gqa_paged_decode_workspace_size(16, 128, 8, 128, 16, 2048, 0, 2) <= 16 << 20
+
+
+def test_measured_split_table():
+    """gqa_pick_splits reads the measured table (nearest cell, units scaled to the device;
+    148 SMs on a host with no GPU), clamped to the pages; num_splits = 0 runs splits only
+    where the sweep found them faster than the balanced schedule."""
+    lib = binding.load()
+    f = lib.gqa_pick_splits
+    assert f(1, 8, 2048, 16, 0) == 16
+    assert f(4, 8, 8192, 16, 0) == 8
+    assert f(64, 8, 2048, 16, 0) == 4
+    assert f(256, 8, 2048, 16, 0) == 1
+    assert f(16, 8, 8192, 16, 1) == 16
+    assert f(1, 8, 100, 16, 0) == 7          # clamped to ceil(100 / 16) pages
+    launches = binding.gqa_paged_decode_kernel_launches
+    assert launches(1, 32, 8, 128, 16, 512, 0, 0) == 2    # auto: 8 splits + lse_combine
+    assert launches(4, 32, 8, 128, 16, 2048, 1, 0) == 2   # e4m3: 8 splits + lse_combine
+    assert launches(64, 32, 8, 128, 16, 2048, 0, 0) == 1  # balanced, in-launch merge
+    assert launches(16, 32, 8, 128, 16, 2048, 0, 0) == 1
+    assert launches(16, 32, 8, 128, 16, 512, 0, -1) == 1  # balanced on request
+    assert launches(16, 32, 8, 128, 16, 512, 0, 0) == 2   # auto: 2 splits + lse_combine
+    # the workspace follows the schedule: splits need their partials
+    ws = lib.gqa_paged_decode_workspace_size
+    assert ws(1, 32, 8, 128, 16, 512, 0, 0) == 256 + (8 * 32 * 128 * 4 + 255) // 256 * 256 + 1024

@@ -2,7 +2,8 @@
 partition among workers, the owner of a tile, and the merge pieces of units that workers
 share.  The formulas are the ones decode_sk_kernel evaluates (restated here): worker W
 owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // per)), per = 16
-tiles, or 4 when T // 16 workers would be under a quarter of them; the owner
+tiles of 16 tokens (8 of 32 tokens), or 4 when T // per workers would be under a quarter of
+them; the owner
 of tile t is ((t+1)*NW + T-1)//T - 1;
 a unit cut between workers leaves one piece per worker, side 1 for the worker where the
 unit begins and side 0 for the others.  The last piece of a unit merges them in the same
@@ -14,8 +15,9 @@ import random
 import pytest
 
 
-def n_workers(workers, T):
-    per = 4 if (T // 16) * 4 < workers else 16
+def n_workers(workers, T, tile_tokens=16):
+    base = 16 * 16 // tile_tokens
+    per = 4 if (T // base) * 4 < workers else base
     return min(workers, max(1, T // per))
 
 
@@ -57,16 +59,18 @@ def schedule(tiles_per_seq, U, workers):
     return T, NW, finals, pieces
 
 
-@pytest.mark.parametrize("workers", [1, 3, 4, 7, 16, 64])
-def test_partition_and_owner(workers):
+@pytest.mark.parametrize("workers,tile_tokens", [(1, 16), (3, 16), (4, 16), (7, 16), (16, 16),
+                                                (64, 16), (4, 32), (16, 32), (64, 32)])
+def test_partition_and_owner(workers, tile_tokens):
+    base = 16 * 16 // tile_tokens
     for T in range(1, 300):
-        NW = n_workers(workers, T)
+        NW = n_workers(workers, T, tile_tokens)
         cover = []
         for W in range(workers):
             cover += list(range(start(W, T, NW), start(W + 1, T, NW)))
         assert cover == list(range(T))
         sizes = [start(W + 1, T, NW) - start(W, T, NW) for W in range(NW)]
-        per = 4 if (T // 16) * 4 < workers else 16
+        per = 4 if (T // base) * 4 < workers else base
         assert max(sizes) - min(sizes) <= 1 and min(sizes) >= min(per, T)
         for t in range(T):
             W = owner(t, T, NW)
