@@ -111,18 +111,21 @@ def tensor_peak():
 
 
 def kernel_src_sha():
+    """Hash of every CUDA source of the library (the kernels a traffic figure belongs to)."""
     h = hashlib.sha256()
-    for rel in ["gqa_attention_paged_b200/csrc/decode.cu", "gqa_attention_paged_b200/csrc/gqa_device.cuh",
-                "gqa_attention_paged_b200/csrc/combine.cu"]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+    csrc = os.path.join(ROOT, "gqa_attention_paged_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_from_profile(workload_key):
-    """DRAM bytes per decode call from the committed ncu summary, or None if absent or
-    taken on a different kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    """DRAM bytes (read + write) per call of the timed kernels, from the committed ncu
+    summary, or None if absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
@@ -527,7 +530,8 @@ def measure_prefill(a, dev, with_cpu):
         "tokens_per_s": round(sum(q_lens) / (ms * 1e-3), 1),
         "spread": spread(more) if more else None,
         "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(tf / peak, 4), "traffic": None,
+                     "frac": round(tf / peak, 4), "traffic": traffic_from_profile("prefill"),
+                     "traffic_key": "prefill",
                      "peak_source": f"{kind} (bf16_tflops, burst cuBLAS GEMM)",
                      "kernel": "prefill_kernel (plan kernel included in the step time)"},
         "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
@@ -850,8 +854,9 @@ def measure_sparse(a, dev, with_cpu):
         "dense_ms_per_step": round(dms, 5), "speedup_over_dense": round(dms / ms, 3),
         "spread": sp,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(gbs / peak, 4), "traffic": None,
-                     "kernel": "sparse_select_kernel + decode_sk_kernel (+ piece merge): the whole call"},
+                     "frac": round(gbs / peak, 4), "traffic": traffic_from_profile("sparse70b"),
+                     "traffic_key": "sparse70b",
+                     "kernel": "sparse_score_kernel + sparse_pick_kernel + decode_sk_kernel (+ piece merge): the whole call"},
         "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hin),
                 "d2h_bytes_per_step": sum(p_[0].numel() * p_[0].element_size() for p_ in hout),
