@@ -111,11 +111,13 @@ def tensor_peak():
 
 
 def kernel_src_sha():
-    """Hash of every CUDA source of the library (the kernels a traffic figure belongs to)."""
+    """Hash of the library's device sources (every file that defines or configures a
+    kernel; the host-only api.cu and static_scratch.cu are left out), the code a traffic
+    figure belongs to."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gqa_attention_paged_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
+        if fn.endswith((".cu", ".cuh", ".h")) and fn not in ("api.cu", "static_scratch.cu"):
             with open(os.path.join(csrc, fn), "rb") as f:
                 h.update(fn.encode())
                 h.update(f.read())
@@ -965,8 +967,8 @@ def run_sweep(kind, a, dev):
                 del inp
                 torch.cuda.empty_cache()
     else:
-        grid = [(B, ctx) for B in (1, 4, 16, 64, 256, 1024) for ctx in (512, 2048, 8192, 32768)
-                if B * ctx <= (2 << 20)]
+        grid = [(B, ctx) for B in (1, 2, 4, 8, 16, 64, 256, 1024)
+                for ctx in (512, 2048, 8192, 32768) if B * ctx <= (2 << 20)]
         for kv in ("bf16", "fp8_e4m3"):
             for B, ctx in grid:
                 inp = device_decode_inputs(B, ctx, Hq, Hk, D, P, kv, dev, seed=B + ctx)

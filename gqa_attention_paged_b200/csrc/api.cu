@@ -75,32 +75,45 @@ bool valid_page_size(int P) { return P == 16 || P == 32 || P == 64; }
 
 int sm_count();
 
-// Split counts measured on one B200 (148 SMs) with `bench.py --sweep splits` (decode_sweep
-// under profiles/): Hq=32, Hk=8, head_dim 128, page 16, every sequence the same length;
-// rows: units B*Hk of 8, 32, 128, 512, 2048, 8192; columns: context 512, 2048, 8192,
-// 32768 tokens; [0] bf16 KV, [1] e4m3 KV.  Cells with B * context above 2M tokens were not
+// Split counts measured on one B200 (148 SMs) with `bench.py --sweep splits` (summary in
+// profiles/decode_sweep_batch_and_splits.md): Hq=32, Hk=8, head_dim 128, page 16, every
+// sequence the same length; rows: units B*Hk (kTabUnitsAt), columns: context in tokens
+// (kTabCtxAt); [0] bf16 KV, [1] e4m3 KV.  Cells with B * context above 2M tokens were not
 // measured and repeat their measured neighbour.
 //   kBestSplits: the split schedule's fastest split count (gqa_pick_splits).
 //   kAutoSplits: what num_splits = 0 runs: 0 = the balanced schedule, else that split
 //     count, where the split schedule measured at least 5% faster than the balanced one
 //     (a few short sequences).
-constexpr int kTabUnits = 6, kTabCtx = 4;
+constexpr int kTabUnits = 8, kTabCtx = 4;
+const int kTabUnitsAt[kTabUnits] = {8, 16, 32, 64, 128, 512, 2048, 8192};
+const int kTabCtxAt[kTabCtx] = {512, 2048, 8192, 32768};
 const unsigned char kBestSplits[2][kTabUnits][kTabCtx] = {
-    {{8, 16, 32, 32}, {4, 8, 8, 32}, {2, 2, 16, 16}, {2, 4, 4, 16}, {1, 1, 4, 4}, {1, 1, 1, 1}},
-    {{8, 16, 32, 32}, {4, 8, 8, 32}, {2, 2, 16, 16}, {1, 4, 4, 16}, {1, 1, 4, 4}, {1, 1, 1, 1}}};
+    {{8, 16, 32, 32}, {8, 16, 16, 16}, {4, 8, 8, 32}, {4, 4, 16, 32}, {2, 2, 16, 16}, {2, 4, 4, 16}, {1, 1, 8, 8}, {1, 1, 1, 1}},
+    {{4, 16, 32, 32}, {8, 8, 16, 16}, {4, 8, 8, 32}, {4, 4, 16, 32}, {2, 2, 16, 16}, {1, 4, 4, 16}, {1, 1, 4, 4}, {1, 1, 1, 1}}};
 const unsigned char kAutoSplits[2][kTabUnits][kTabCtx] = {
-    {{8, 0, 0, 0}, {4, 8, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}},
-    {{8, 16, 0, 0}, {4, 8, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}}};
+    {{8, 0, 0, 0}, {8, 0, 16, 0}, {4, 8, 0, 0}, {4, 4, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}},
+    {{4, 16, 0, 0}, {8, 8, 0, 0}, {4, 8, 0, 0}, {4, 4, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}}};
 
-// Table cell of (units, context): the nearest row and column in log scale (rows and
-// columns are a factor 4 apart); units are first scaled to 148 SMs.
+// Index of the entry of `at` nearest to x in log scale.
+int nearest_log(const int *at, int n, double x) {
+    int best = 0;
+    double bd = 1e30;
+    const double lx = log(x > 1.0 ? x : 1.0);
+    for (int i = 0; i < n; ++i) {
+        const double d = fabs(log((double)at[i]) - lx);
+        if (d < bd) {
+            bd = d;
+            best = i;
+        }
+    }
+    return best;
+}
+
+// Table cell of (units, context); units are first scaled to 148 SMs.
 void split_cell(int B, int Hk, int max_seq_len, int &ui, int &ci) {
-    double units = (double)B * Hk * 148.0 / (double)sm_count();
-    double ctx = max_seq_len > 0 ? (double)max_seq_len : 1.0;
-    int u = (int)lround(log(units / 8.0) / log(4.0));
-    int c = (int)lround(log(ctx / 512.0) / log(4.0));
-    ui = u < 0 ? 0 : (u >= kTabUnits ? kTabUnits - 1 : u);
-    ci = c < 0 ? 0 : (c >= kTabCtx ? kTabCtx - 1 : c);
+    const double units = (double)B * Hk * 148.0 / (double)sm_count();
+    ui = nearest_log(kTabUnitsAt, kTabUnits, units);
+    ci = nearest_log(kTabCtxAt, kTabCtx, (double)max_seq_len);
 }
 
 int clamp_splits(int s, int max_seq_len, int P) {
