@@ -110,33 +110,41 @@ def tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_src_sha():
-    """Hash of the library's device sources (every file that defines or configures a
-    kernel; the host-only api.cu and static_scratch.cu are left out), the code a traffic
+# Device sources behind each workload's kernels (the shared device headers included).
+SRC_COMMON = ("gqa_device.cuh", "gqa_internal.h")
+SRC_OF = {"decode": ("decode.cu", "combine.cu"), "prefill": ("prefill.cu",),
+          "sparse": ("sparse.cu", "decode.cu", "combine.cu")}
+
+
+def src_family(workload_key):
+    return "prefill" if workload_key == "prefill" else "sparse" if workload_key.startswith("sparse") else "decode"
+
+
+def kernel_src_sha(workload_key="B64_ctx2048_bf16_S0_pack1"):
+    """Hash of the device sources a workload's kernels are built from: the code a traffic
     figure belongs to."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gqa_attention_paged_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")) and fn not in ("api.cu", "static_scratch.cu"):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    for fn in sorted(SRC_COMMON + SRC_OF[src_family(workload_key)]):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_from_profile(workload_key):
     """DRAM bytes (read + write) per call of the timed kernels, from the committed ncu
-    summary, or None if absent or taken on a different kernel source."""
+    summary, or None if absent or taken on different kernel sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("kernel_src_sha") != kernel_src_sha():
-        return None
     e = d.get("workloads", {}).get(workload_key)
-    return None if e is None else float(e["dram_bytes_per_launch"])
+    if e is None or e.get("kernel_src_sha") != kernel_src_sha(workload_key):
+        return None
+    return float(e["dram_bytes_per_launch"])
 
 
 # ------------------------------------------------------------------------ clocks

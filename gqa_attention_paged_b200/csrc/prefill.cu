@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(1024)
         if (c >= 0) atomicAdd(&hist[c], 1);
         if (idx % items_per_seq == 0) {
             const int b = idx / items_per_seq;
-            if (a.cu_q[b + 1] - a.cu_q[b] > items_per_seq * 2 * T)
+            if (a.cu_q[b + 1] - a.cu_q[b] > a.max_q_len)
                 set_error(a.err, GQA_ERR_SHAPE);  // max_q_len below a chunk length
         }
     }
