@@ -835,6 +835,10 @@ def measure_sparse(a, dev, with_cpu):
     e2e_ms = e2e_pipelined(dev, stream, hin, din, dout, hout, run, a.steps)
     peak, kind = peaks()
     gbs = step_bytes / (ms * 1e-3) / 1e9
+    # the decode of the chosen pages: B * Hk sequences of one kv head and Hq / Hk heads
+    dec_launches = binding.gqa_paged_decode_kernel_launches(
+        B * Hk, Hq // Hk, 1, D, P, binding.gqa_paged_sparse_table_stride(pt.shape[1], P, topk, window) * P,
+        0, 0)
     cpu = None
     if with_cpu:
         from oracle import oracle
@@ -866,14 +870,13 @@ def measure_sparse(a, dev, with_cpu):
         "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "traffic": traffic_from_profile("sparse70b"),
                      "traffic_key": "sparse70b",
-                     "kernel": "sparse_score_kernel + sparse_pick_kernel + decode_sk_kernel (+ piece merge): the whole call"},
+                     "kernel": "sparse_score_kernel + sparse_pick_kernel + the decode of the chosen pages as "
+                               f"num_splits = 0 schedules it ({dec_launches} launch(es)): the whole call"},
         "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hin),
                 "d2h_bytes_per_step": sum(p_[0].numel() * p_[0].element_size() for p_ in hout),
                 "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": a.steps * (1 + binding.gqa_paged_decode_kernel_launches(
-            B * Hk, Hq // Hk, 1, D, P, binding.gqa_paged_sparse_table_stride(pt.shape[1], P, topk, window) * P,
-            0, 0)),
+        "gpu_launches": a.steps * (2 + dec_launches),
         "clocks": clk, "cpu_baseline": cpu,
     }
 

@@ -1178,7 +1178,9 @@ cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtenso
         const size_t smem =
             sizeof(Smem<D, FP8, kRingBalanced, TT>) + 1024 + sizeof(int) * (size_t)(a.B + 1);
         const bool defer = decode_defers_merge(a.B, a.Hq, a.Hk, a.pack_gqa, a.grid);
-        auto kern = defer ? decode_sk_kernel<D, NT, FP8, TT, true> : decode_sk_kernel<D, NT, FP8, TT, false>;
+        // the 16-head instance (NT = 2) always defers (decode_defers_merge): it has no
+        // in-launch-merge instance
+        auto kern = defer ? decode_sk_kernel<D, NT, FP8, TT, true> : decode_sk_kernel<D, NT, FP8, TT, NT == 2>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         // programmatic stream serialization: the kernel's set-up overlaps the tail of the

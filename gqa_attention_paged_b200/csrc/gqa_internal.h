@@ -53,10 +53,14 @@ inline int decode_heads_per_cta(int Hq, int Hk, int pack_gqa) {
 }
 // A balanced-schedule launch whose units average more than this many workers each leaves
 // its pieces to a second kernel, which merges every cut unit in parallel; otherwise the
-// last piece of each unit merges the unit in the same launch.
+// last piece of each unit merges the unit in the same launch.  The 16-head instance
+// (groups above 8) always leaves them: with the merge in the same launch its streaming
+// loop spills, and it measured 1.3-1.9x slower at B=64 (Hq/Hk = 32/2 and 64/4) and no
+// faster anywhere.
 constexpr int kDeferMinWorkersPerUnit = 24;
 inline bool decode_defers_merge(int B, int Hq, int Hk, int pack_gqa, int grid) {
     const int g = Hq / Hk, hpc = decode_heads_per_cta(Hq, Hk, pack_gqa);
+    if (hpc > 8) return true;
     const long long units = (long long)B * Hk * ((g + hpc - 1) / hpc);
     return (long long)grid * kStreamWorkersPerCta > (long long)kDeferMinWorkersPerUnit * units;
 }

@@ -202,6 +202,7 @@ def test_measured_split_table():
     assert launches(16, 32, 8, 128, 16, 2048, 0, 0) == 1
     assert launches(16, 32, 8, 128, 16, 512, 0, -1) == 1  # balanced on request
     assert launches(16, 32, 8, 128, 16, 512, 0, 0) == 2   # auto: 2 splits + lse_combine
+    assert launches(64, 32, 2, 128, 16, 2048, 0, 0) == 2  # groups of 16: decode + merge kernel
     # the workspace follows the schedule: splits need their partials
     ws = lib.gqa_paged_decode_workspace_size
     assert ws(1, 32, 8, 128, 16, 512, 0, 0) == 256 + (8 * 32 * 128 * 4 + 255) // 256 * 256 + 1024

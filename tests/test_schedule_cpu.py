@@ -125,6 +125,8 @@ def defers(B, Hq, Hk, pack, grid):
     leave their pieces to the separate merge kernel."""
     g = Hq // Hk
     hpc = (min(g, 16 if g > 8 else 8)) if pack else 1
+    if hpc > 8:
+        return True  # the 16-head instance always leaves its pieces to the merge kernel
     units = B * Hk * ((g + hpc - 1) // hpc)
     return grid * 4 > 24 * units
 
@@ -176,3 +178,5 @@ def test_defer_policy_on_the_named_shapes():
     assert not defers(64, 32, 8, True, grid)   # B=64 sweep: 2 workers per unit
     assert not defers(16, 32, 8, True, grid)   # 7B-shaped batch
     assert not defers(8, 32, 8, False, grid)   # PackGQA off: one unit per head
+    assert defers(64, 32, 2, True, grid)       # groups of 16: always the merge kernel
+    assert not defers(64, 32, 2, False, grid)  # ... unless PackGQA is off
