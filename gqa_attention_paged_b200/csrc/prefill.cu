@@ -22,8 +22,8 @@
 //               MMAs from one thread in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so the
 //               tensor core works on one query tile while the other one's softmax runs.
 //   warps 2-3   load the V tiles (warp 2, the same way) and convert each in place from
-//               bf16 to f16 (zeroing keys past the sequence first), unless a value is
-//               beyond the f16 range.
+//               bf16 to f16, keys past the sequence zeroed first; a tile with a value
+//               beyond the f16 range is copied again and stays bf16.
 //   warps 4-7   softmax of query tile 0, warps 8-11 of query tile 1; a thread owns one
 //               row (one tensor-memory lane) and holds its 128 scores in registers.
 // The softmax warpgroups take most of the register file (setmaxnreg).
@@ -64,8 +64,6 @@ constexpr int kRegsSide = 64;
 constexpr int kRegsSoftmax = 216;
 static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreadsP * 168, "register split");
 constexpr int kConvThreads = 64;
-// |bf16 bits| at or above this (2^16, and Inf / NaN) does not convert to a finite f16
-constexpr uint32_t kF16Limit = 0x4780u;
 
 template <int D>
 struct alignas(1024) PSmem {
@@ -77,6 +75,7 @@ struct alignas(1024) PSmem {
     uint64_t v_full[kVStages], v_ready[kVStages], v_empty[kVStages];
     uint64_t s_full[kQT], p_full[kQT], pv_done[kQT];
     uint64_t mma_done;
+    uint64_t v_fixsync, v_fix;  // a V tile out of f16 range: both converters done, copied again
     int v_bf16[kVStages];       // 1: the V tile stayed bf16 (a value out of f16 range)
     int conv_ovf[kVStages][2];  // per converter warp: (tile + 1) * 2 + out-of-range flag
     uint32_t tmem_base;
@@ -400,6 +399,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             mbar_init(&sm.pv_done[q], 1);
         }
         mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.v_fixsync, 2);
+        mbar_init(&sm.v_fix, 1);
         for (int s = 0; s < kVStages; ++s) sm.conv_ovf[s][0] = sm.conv_ovf[s][1] = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -552,20 +553,25 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         const int32_t *pt = a.page_table + (size_t)b * a.pt_stride;
         const uint64_t pol_kv = policy_evict_last();
         int issued_v = 0;
-        auto load_v = [&](int jv) {
+        // V tile jv into its stage, counted on `bar`
+        auto load_v_to = [&](int jv, uint64_t *bar) {
             const int row = kv_chunk_row(a, pt, jv, lane, kvh, L);
             const unsigned mask = __ballot_sync(kAll, row >= 0);
             const int vs = jv % kVStages;
-            if (lane == 0) mbar_arrive_expect_tx(&sm.v_full[vs], __popc(mask) * kHalves * kChunkBytes);
+            if (lane == 0) mbar_arrive_expect_tx(bar, __popc(mask) * kHalves * kChunkBytes);
             __syncwarp();
             if (row >= 0) {
 #pragma unroll
                 for (int h = 0; h < kHalves; ++h)
-                    tma_load_2d(sm.v[vs] + h * kHalfBytes + lane * kChunkBytes, &vmap,
-                                &sm.v_full[vs], 64 * h, row, pol_kv);
+                    tma_load_2d(sm.v[vs] + h * kHalfBytes + lane * kChunkBytes, &vmap, bar, 64 * h, row,
+                                pol_kv);
             }
+        };
+        auto load_v = [&](int jv) {
+            load_v_to(jv, &sm.v_full[jv % kVStages]);
             issued_v = jv + 1;
         };
+        int nfix = 0;  // V tiles copied again so far (the same count in both converter warps)
         if (cw == 0)
             for (int jv = 0; jv < min(n_kv, kVStages); ++jv) load_v(jv);
         for (int j = 0; j < n_kv; ++j) {
@@ -576,11 +582,18 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             }
             uint8_t *vt = sm.v[stage];
             // Each thread owns chunks cid, cid + 64, ... (chunk c: half c / 1024, key row
-            // (c / 8) % 128) through both passes, so no other thread touches them.
-            // pass 1: keys at or past L hold anything (even NaN): zero those rows so their
-            // zero weights contribute exactly zero (zero has the same bits in bf16 and f16);
-            // find the largest magnitude (as bf16 bits) of the rest.
+            // (c / 8) % 128).  On the sequence's last tile the keys at or past L (which hold
+            // anything, even NaN) become zero first, so their zero weights add exactly zero
+            // (zero has the same bits in bf16 and f16).  Then every chunk becomes f16 in place
+            // (bf16 -> fp32 is exact; fp32 -> f16 rounds to nearest, magnitudes under 2^-14
+            // becoming f16 subnormals).  A value beyond the f16 range (or Inf / NaN) comes out
+            // with all exponent bits set: the largest magnitude of the results shows it.
             const int valid = L - j * kN;
+            if (valid < kN) {
+                for (int c = cid; c < kChunks16; c += kConvThreads)
+                    if (((c >> 3) & (kN - 1)) >= valid)
+                        *reinterpret_cast<uint4 *>(vt + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+            }
             uint32_t mx = 0u;
             constexpr int kBatch = 8;  // chunks in flight per thread
 #pragma unroll 1
@@ -591,16 +604,16 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     w[i] = *reinterpret_cast<const uint4 *>(vt + 16 * (c0 + i * kConvThreads));
 #pragma unroll
                 for (int i = 0; i < kBatch; ++i) {
-                    const int c = c0 + i * kConvThreads;
-                    if (((c >> 3) & (kN - 1)) >= valid) {
-                        *reinterpret_cast<uint4 *>(vt + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
-                    } else {
-                        mx = umax16x2(mx, umax16x2(umax16x2(w[i].x & 0x7fff7fffu, w[i].y & 0x7fff7fffu),
-                                                   umax16x2(w[i].z & 0x7fff7fffu, w[i].w & 0x7fff7fffu)));
-                    }
+                    w[i].x = pack_f16(__uint_as_float(w[i].x << 16), __uint_as_float(w[i].x & 0xffff0000u));
+                    w[i].y = pack_f16(__uint_as_float(w[i].y << 16), __uint_as_float(w[i].y & 0xffff0000u));
+                    w[i].z = pack_f16(__uint_as_float(w[i].z << 16), __uint_as_float(w[i].z & 0xffff0000u));
+                    w[i].w = pack_f16(__uint_as_float(w[i].w << 16), __uint_as_float(w[i].w & 0xffff0000u));
+                    mx = umax16x2(mx, umax16x2(umax16x2(w[i].x & 0x7fff7fffu, w[i].y & 0x7fff7fffu),
+                                               umax16x2(w[i].z & 0x7fff7fffu, w[i].w & 0x7fff7fffu)));
+                    *reinterpret_cast<uint4 *>(vt + 16 * (c0 + i * kConvThreads)) = w[i];
                 }
             }
-            const bool big = (mx & 0xffffu) >= kF16Limit || (mx >> 16) >= kF16Limit;
+            const bool big = (mx & 0xffffu) >= 0x7c00u || (mx >> 16) >= 0x7c00u;
             // exchange the range decision with the other converter warp: (j + 1) * 2 + flag, and a
             // bounded wait for the partner's entry of this tile
             const int mine = ((j + 1) << 1) | (__any_sync(kAll, big) ? 1 : 0);
@@ -616,24 +629,28 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 break;
             }
             const bool keep_bf16 = ((mine | theirs) & 1) != 0;
-            if (!keep_bf16) {
-                // pass 2: bf16 -> f16 in place (bf16 -> fp32 is exact; fp32 -> f16 rounds
-                // to nearest, magnitudes under 2^-14 becoming f16 subnormals)
-#pragma unroll 1
-                for (int c0 = cid; c0 < kChunks16; c0 += kBatch * kConvThreads) {
-                    uint4 w[kBatch];
-#pragma unroll
-                    for (int i = 0; i < kBatch; ++i)
-                        w[i] = *reinterpret_cast<const uint4 *>(vt + 16 * (c0 + i * kConvThreads));
-#pragma unroll
-                    for (int i = 0; i < kBatch; ++i) {
-                        w[i].x = pack_f16(__uint_as_float(w[i].x << 16), __uint_as_float(w[i].x & 0xffff0000u));
-                        w[i].y = pack_f16(__uint_as_float(w[i].y << 16), __uint_as_float(w[i].y & 0xffff0000u));
-                        w[i].z = pack_f16(__uint_as_float(w[i].z << 16), __uint_as_float(w[i].z & 0xffff0000u));
-                        w[i].w = pack_f16(__uint_as_float(w[i].w << 16), __uint_as_float(w[i].w & 0xffff0000u));
-                        *reinterpret_cast<uint4 *>(vt + 16 * (c0 + i * kConvThreads)) = w[i];
-                    }
+            if (keep_bf16) {
+                // Copy tile j again (bf16) once both warps' f16 stores are ordered before the
+                // copy: each warp fences them for the async proxy and arrives on v_fixsync, and
+                // warp 2 issues the copy after both arrivals.  Then the keys past L become zero
+                // again.
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.v_fixsync);
+                bool fixed = true;
+                if (cw == 0) {
+                    fixed = wait_all(&sm.v_fixsync, nfix & 1);
+                    if (fixed) load_v_to(j, &sm.v_fix);
                 }
+                if (!fixed || !wait_all(&sm.v_fix, nfix & 1)) {
+                    if (lane == 0) set_error(a.err, GQA_ERR_TIMEOUT);
+                    break;
+                }
+                ++nfix;
+                if (valid < kN)
+                    for (int c = cid; c < kChunks16; c += kConvThreads)
+                        if (((c >> 3) & (kN - 1)) >= valid)
+                            *reinterpret_cast<uint4 *>(vt + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
             }
             // the tensor core (async proxy) reads what these generic stores wrote
             fence_proxy_async_smem();
