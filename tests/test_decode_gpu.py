@@ -257,7 +257,7 @@ def test_chained_decodes_read_the_previous_output():
 def test_decode_replays_in_a_cuda_graph(lens):
     """The balanced schedule captured in a CUDA graph (both merge variants: in-launch for
     many short units, the separate merge kernel for two long sequences) replays to the
-    eager result, bit for bit."""
+    oracle's result within the bf16 gate, and to the eager result bit for bit."""
     case = inputs.make_decode_case(len(lens), 32, 8, 128, 16, lens, seed=21)
     d = to_dev(case)
     B = len(lens)
@@ -281,6 +281,8 @@ def test_decode_replays_in_a_cuda_graph(lens):
     g.replay()
     torch.cuda.synchronize()
     assert binding.gqa_get_error(ws) == 0
+    ref_o, ref_l = oracle_decode(case)
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, what=f"graph replay {lens[:2]}")
     assert torch.equal(out, eager_o) and torch.equal(lse, eager_l)
     del g
 
