@@ -83,7 +83,8 @@ def test_sweep_decode_batch(B):
     rows = np.arange(B) if B <= 16 else np.sort(np.random.default_rng(B).choice(B, 8, replace=False))
     ref_o, ref_l = _sampled_oracle(case, rows)
     dev = to_dev(case)
-    for S in ([0, 1, 2, 4] if B in (1, 64) else [0]):
+    # num_splits 0 (the measured choice), the balanced schedule on request, and splits
+    for S in ([0, binding.GQA_SPLITS_BALANCED, 1, 2, 4] if B in (1, 64) else [0]):
         out, lse = run_decode(case, num_splits=S, dev=dev)
         check(out[rows], lse[rows], ref_o, ref_l, what=f"sweep B={B} S={S}")
 
@@ -121,14 +122,16 @@ def test_long70b_decode_fp8(S):
 @pytest.mark.parametrize("P", [16, 32, 64])
 @pytest.mark.parametrize("Hq,Hk", [(32, 8), (64, 8), (8, 8)])
 def test_fp8_page_sizes_and_ragged_tiles(P, Hq, Hk):
-    """e4m3 KV takes 32-token tiles on pages of 32+ tokens: lengths that end inside either
-    16-token half of a tile, exactly on a tile edge, empty, and longer than a page."""
+    """e4m3 KV takes 32-token tiles on pages of 32+ tokens (and in the balanced schedule on
+    any page): lengths that end inside either 16-token half of a tile, exactly on a tile
+    edge, empty, and longer than a page; num_splits 0 (here the measured split count), the
+    balanced schedule on request, splits, and PackGQA off."""
     lens = [1, 15, 16, 17, 31, 32, 33, 0, 63, 200]
     case = inputs.make_decode_case(len(lens), Hq, Hk, 128, P, lens, seed=P + Hq,
                                    kv_dtype="fp8_e4m3", outlier_p=0.01)
     ref_o, ref_l = oracle_decode(case)
     dev = to_dev(case)
-    for S, pack in ((0, True), (1, True), (3, True), (1, False)):
+    for S, pack in ((0, True), (binding.GQA_SPLITS_BALANCED, True), (1, True), (3, True), (1, False)):
         out, lse = run_decode(case, num_splits=S, pack_gqa=pack, dev=dev)
         check(out, lse, ref_o, ref_l, what=f"fp8 P={P} Hq={Hq} S={S} pack={pack}")
 
@@ -138,7 +141,7 @@ def test_fp8_page_sizes_and_ragged_tiles(P, Hq, Hk):
 def test_head_layouts_mha_mqa_and_odd_groups(Hq, Hk, D, P):
     case = inputs.make_decode_case(3, Hq, Hk, D, P, [1, 150, 333], seed=Hq * D + P)
     ref_o, ref_l = oracle_decode(case)
-    for S in (0, 1, 3):
+    for S in (0, binding.GQA_SPLITS_BALANCED, 1, 3):
         out, lse = run_decode(case, num_splits=S)
         check(out, lse, ref_o, ref_l, what=f"Hq={Hq} Hk={Hk} D={D} P={P} S={S}")
 
@@ -146,7 +149,7 @@ def test_head_layouts_mha_mqa_and_odd_groups(Hq, Hk, D, P):
 def test_empty_and_single_token_sequences():
     case = inputs.make_decode_case(5, 8, 2, 128, 16, [0, 1, 0, 16, 17], seed=21)
     ref_o, ref_l = oracle_decode(case)
-    for S in (0, 1, 2, 5):
+    for S in (0, binding.GQA_SPLITS_BALANCED, 1, 2, 5):
         out, lse = run_decode(case, num_splits=S)
         check(out, lse, ref_o, ref_l, what=f"empty S={S}")
         assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
