@@ -64,7 +64,7 @@ def _simulate(case, world, S):
 
 
 @pytest.mark.parametrize("world", [1, 2, 3, 4])
-@pytest.mark.parametrize("S", [0, 3])
+@pytest.mark.parametrize("S", [0, binding.GQA_SPLITS_BALANCED, 3])
 def test_split_ranks_llama7b(world, S):
     case = inputs.llama7b_decode(seed=31)
     out, lse = _simulate(case, world, S)
