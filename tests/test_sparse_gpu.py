@@ -120,6 +120,15 @@ def test_selection_is_bit_exact(name, topk, window):
     _check_selection(case, _dev(case), topk, window)
 
 
+@pytest.mark.parametrize("topk,window", [(4, 32), (300, 16)])
+def test_selection_is_bit_exact_on_a_table_of_more_than_1024_pages(topk, window):
+    """A table of 1250 pages of 16 tokens: more pages than the pick's 512 threads, so each
+    thread takes several pages in every radix pass, count and compaction."""
+    case = inputs.make_decode_case(2, 16, 2, 128, 16, [20000, 5000], seed=48)
+    assert case.kv.page_table.shape[1] > 1024
+    _check_selection(case, _dev(case), topk, window)
+
+
 def test_selection_ties_go_to_the_lower_page():
     case = inputs.make_decode_case(2, 32, 8, 128, 16, [320, 200], seed=47, pt_stride=20)
     pt = case.kv.page_table.clone()
