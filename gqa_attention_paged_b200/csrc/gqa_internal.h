@@ -53,11 +53,13 @@ inline int decode_heads_per_cta(int Hq, int Hk, int pack_gqa) {
 }
 // A balanced-schedule launch whose units average more than this many workers each leaves
 // its pieces to a second kernel, which merges every cut unit in parallel; otherwise the
-// last piece of each unit merges the unit in the same launch.  The 16-head instance
+// last piece of each unit merges the unit in the same launch, reading the unit's pieces
+// one after another.  Measured at ctx 2048: 9 workers per unit (B=16) 32.8 -> 29.8 us
+// with the second kernel, 4.6 (B=32) no gain, 2.3 (B=64) 91.9 -> 100.7 us.  The 16-head instance
 // (groups above 8) always leaves them: with the merge in the same launch its streaming
 // loop spills, and it measured 1.3-1.9x slower at B=64 (Hq/Hk = 32/2 and 64/4) and no
 // faster anywhere.
-constexpr int kDeferMinWorkersPerUnit = 24;
+constexpr int kDeferMinWorkersPerUnit = 8;
 inline bool decode_defers_merge(int B, int Hq, int Hk, int pack_gqa, int grid) {
     const int g = Hq / Hk, hpc = decode_heads_per_cta(Hq, Hk, pack_gqa);
     if (hpc > 8) return true;

@@ -92,7 +92,7 @@ size_t gqa_paged_decode_workspace_size(int B, int Hq, int Hk, int head_dim, int 
 /*
  * Kernels one gqa_paged_decode() call with these arguments launches on the current
  * device: 1, or 2 when a second kernel merges partial results (split schedule with
- * S > 1: lse_combine; balanced schedule when its units average more than 24 workers
+ * S > 1: lse_combine; balanced schedule when its units average more than 8 workers
  * each, e.g. a few long sequences: the kernel that merges the pieces of cut units).
  * Returns 0 for sizes gqa_paged_decode() rejects.  Host only; launches nothing.
  */

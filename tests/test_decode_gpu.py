@@ -215,9 +215,10 @@ def test_lse_combine_standalone():
     assert np.isneginf(lse[3]) and np.all(out[3] == 0)
 
 
-@pytest.mark.parametrize("B,S", [(16, 0), (4, 3), (4, 0)])
+@pytest.mark.parametrize("B,S", [(48, 0), (16, 0), (4, 3), (4, 0)])
 def test_repeated_calls_are_deterministic(B, S):
-    """B=16 with num_splits=0 runs the balanced schedule; B=4 at context 2048 with
+    """B=48 with num_splits=0 runs the balanced schedule with the in-launch merge, B=16
+    the balanced schedule with the separate merge kernel; B=4 at context 2048 with
     num_splits=0 runs the measured split count (a small problem)."""
     case = inputs.llama7b_decode(seed=6, B=B)
     dev = to_dev(case)
@@ -225,7 +226,7 @@ def test_repeated_calls_are_deterministic(B, S):
     a = run_decode(case, num_splits=S, dev=dev, workspace=ws)
     b = run_decode(case, num_splits=S, dev=dev, workspace=ws)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
-    if B == 16 and S == 0:  # balanced: merge counters are back to zero after every launch
+    if B == 48 and S == 0:  # in-launch merge: counters are back to zero after every launch
         hdr = 256
         assert binding.gqa_paged_decode_kernel_launches(B, 32, 8, 128, 16, 2048, 0, 0) == 1
         assert int(ws[hdr:hdr + B * 32 * 4].view(torch.int32).abs().sum()) == 0

@@ -121,14 +121,14 @@ def test_slot_indices_stay_in_the_workspace():
 
 
 def defers(B, Hq, Hk, pack, grid):
-    """The host policy (decode_defers_merge): units averaging more than 24 workers each
+    """The host policy (decode_defers_merge): units averaging more than 8 workers each
     leave their pieces to the separate merge kernel."""
     g = Hq // Hk
     hpc = (min(g, 16 if g > 8 else 8)) if pack else 1
     if hpc > 8:
         return True  # the 16-head instance always leaves its pieces to the merge kernel
     units = B * Hk * ((g + hpc - 1) // hpc)
-    return grid * 4 > 24 * units
+    return grid * 4 > 8 * units
 
 
 def merge_kernel_reads(tiles_per_seq, U, workers):
@@ -176,7 +176,8 @@ def test_defer_policy_on_the_named_shapes():
     assert defers(4, 64, 8, True, grid)        # 70B long context: 32 units, 37 workers each
     assert defers(1, 32, 8, True, grid)        # one sequence
     assert not defers(64, 32, 8, True, grid)   # B=64 sweep: 2 workers per unit
-    assert not defers(16, 32, 8, True, grid)   # 7B-shaped batch
+    assert defers(16, 32, 8, True, grid)       # 7B-shaped batch: 9 workers per unit
+    assert not defers(32, 32, 8, True, grid)   # 4.6 workers per unit
     assert not defers(8, 32, 8, False, grid)   # PackGQA off: one unit per head
     assert defers(64, 32, 2, True, grid)       # groups of 16: always the merge kernel
     assert not defers(64, 32, 2, False, grid)  # ... unless PackGQA is off

@@ -85,12 +85,12 @@ def test_static_scratch_balanced_after_split_calls():
     """split (S=4) -> balanced -> balanced with the separate piece merge -> balanced again.
     The first balanced call's merge counters occupy bytes the split call's partials
     overwrote, so they must be cleared by the call itself."""
-    ragged = inputs.llama7b_decode(seed=21)
+    ragged = inputs.llama7b_decode(seed=21, B=48)
     few_long = inputs.make_decode_case(2, 32, 8, 128, 16, [4096, 3001], seed=22)
     d_r, d_f = _dev(ragged), _dev(few_long)
     # the second balanced shape really takes the separate piece merge
     assert binding.gqa_paged_decode_kernel_launches(2, 32, 8, 128, 16, 4096, 0, 0) == 2
-    assert binding.gqa_paged_decode_kernel_launches(16, 32, 8, 128, 16, 2048, 0, 0) == 1
+    assert binding.gqa_paged_decode_kernel_launches(48, 32, 8, 128, 16, 2048, 0, 0) == 1
     _check(ragged, d_r, 4, "split S=4")
     o1, l1 = _check(ragged, d_r, 0, "balanced after split")
     _check(few_long, d_f, 0, "balanced, separate piece merge")
