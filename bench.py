@@ -979,7 +979,7 @@ def run_sweep(kind, a, dev):
                 torch.cuda.empty_cache()
     else:
         grid = [(B, ctx) for B in (1, 2, 4, 8, 16, 64, 256, 1024)
-                for ctx in (512, 2048, 8192, 32768) if B * ctx <= (2 << 20)]
+                for ctx in (512, 2048, 4096, 8192, 32768) if B * ctx <= (2 << 20)]
         for kv in ("bf16", "fp8_e4m3"):
             for B, ctx in grid:
                 inp = device_decode_inputs(B, ctx, Hq, Hk, D, P, kv, dev, seed=B + ctx)

@@ -75,24 +75,24 @@ bool valid_page_size(int P) { return P == 16 || P == 32 || P == 64; }
 
 int sm_count();
 
-// Split counts measured on one B200 (148 SMs) with `bench.py --sweep splits` (summary in
-// profiles/decode_sweep_batch_and_splits.md): Hq=32, Hk=8, head_dim 128, page 16, every
-// sequence the same length; rows: units B*Hk (kTabUnitsAt), columns: context in tokens
-// (kTabCtxAt); [0] bf16 KV, [1] e4m3 KV.  Cells with B * context above 2M tokens were not
-// measured and repeat their measured neighbour.
+// Split counts measured on one B200 (148 SMs) with `bench.py --sweep splits` (its summary is
+// committed under profiles/): Hq=32, Hk=8, head_dim 128, page 16, every sequence the same
+// length; rows: units B*Hk (kTabUnitsAt), columns: context in tokens (kTabCtxAt); [0] bf16
+// KV, [1] e4m3 KV.  Cells with B * context above 2M tokens were not measured and repeat
+// their measured neighbour.
 //   kBestSplits: the split schedule's fastest split count (gqa_pick_splits).
 //   kAutoSplits: what num_splits = 0 runs: 0 = the balanced schedule, else that split
 //     count, where the split schedule measured at least 5% faster than the balanced one
 //     (a few short sequences).
-constexpr int kTabUnits = 8, kTabCtx = 4;
+constexpr int kTabUnits = 8, kTabCtx = 5;
 const int kTabUnitsAt[kTabUnits] = {8, 16, 32, 64, 128, 512, 2048, 8192};
-const int kTabCtxAt[kTabCtx] = {512, 2048, 8192, 32768};
+const int kTabCtxAt[kTabCtx] = {512, 2048, 4096, 8192, 32768};
 const unsigned char kBestSplits[2][kTabUnits][kTabCtx] = {
-    {{8, 16, 32, 32}, {8, 16, 16, 16}, {4, 8, 8, 32}, {4, 4, 16, 32}, {2, 2, 16, 16}, {2, 4, 4, 16}, {1, 1, 8, 8}, {1, 1, 1, 1}},
-    {{4, 16, 32, 32}, {8, 8, 16, 16}, {4, 8, 8, 32}, {4, 4, 16, 32}, {2, 2, 16, 16}, {1, 4, 4, 16}, {1, 1, 4, 4}, {1, 1, 1, 1}}};
+    {{8, 16, 16, 32, 32}, {8, 16, 16, 16, 16}, {4, 8, 8, 8, 32}, {4, 4, 4, 16, 32}, {2, 2, 8, 16, 16}, {2, 4, 4, 4, 8}, {1, 1, 1, 1, 1}, {1, 1, 1, 1, 1}},
+    {{4, 16, 16, 32, 32}, {8, 8, 16, 16, 16}, {4, 8, 8, 8, 32}, {4, 4, 4, 16, 32}, {2, 2, 8, 16, 16}, {1, 4, 4, 4, 16}, {1, 1, 1, 4, 4}, {1, 1, 1, 1, 1}}};
 const unsigned char kAutoSplits[2][kTabUnits][kTabCtx] = {
-    {{8, 0, 0, 0}, {8, 0, 16, 0}, {4, 8, 0, 0}, {4, 4, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}},
-    {{4, 16, 0, 0}, {8, 8, 0, 0}, {4, 8, 0, 0}, {4, 4, 0, 0}, {2, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}}};
+    {{8, 0, 0, 0, 0}, {8, 0, 0, 16, 0}, {4, 0, 8, 0, 0}, {4, 4, 0, 0, 0}, {2, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}},
+    {{4, 16, 0, 0, 0}, {8, 8, 0, 0, 0}, {4, 8, 8, 0, 0}, {4, 4, 0, 0, 0}, {2, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}}};
 
 // Index of the entry of `at` nearest to x in log scale.
 int nearest_log(const int *at, int n, double x) {

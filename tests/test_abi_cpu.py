@@ -207,4 +207,8 @@ def test_measured_split_table():
     assert launches(64, 32, 2, 128, 16, 2048, 0, 0) == 2  # groups of 16: decode + merge kernel
     # the workspace follows the schedule: splits need their partials
     ws = lib.gqa_paged_decode_workspace_size
+    # B=8: 4 splits at context 2048, the balanced schedule from context 4096 on
+    assert ws(8, 32, 8, 128, 16, 2048, 0, 0) == ws(8, 32, 8, 128, 16, 2048, 0, 4)
+    assert ws(8, 32, 8, 128, 16, 4096, 0, 0) == ws(8, 32, 8, 128, 16, 4096, 0, -1)
+    assert ws(8, 32, 8, 128, 16, 4096, 0, 0) != ws(8, 32, 8, 128, 16, 4096, 0, 4)
     assert ws(1, 32, 8, 128, 16, 512, 0, 0) == 256 + (8 * 32 * 128 * 4 + 255) // 256 * 256 + 1024

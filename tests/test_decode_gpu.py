@@ -218,8 +218,8 @@ def test_lse_combine_standalone():
 @pytest.mark.parametrize("B,S", [(48, 0), (16, 0), (4, 3), (4, 0)])
 def test_repeated_calls_are_deterministic(B, S):
     """B=48 with num_splits=0 runs the balanced schedule with the in-launch merge, B=16
-    the balanced schedule with the separate merge kernel; B=4 at context 2048 with
-    num_splits=0 runs the measured split count (a small problem)."""
+    and B=4 the balanced schedule with the separate merge kernel; B=4 with 3 splits the
+    split schedule and lse_combine."""
     case = inputs.llama7b_decode(seed=6, B=B)
     dev = to_dev(case)
     ws = binding.new_workspace(binding.gqa_paged_decode_workspace_size(B, 32, 8, 128, 16, 2048, 0, S), DEV)
