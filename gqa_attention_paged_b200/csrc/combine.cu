@@ -19,6 +19,9 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float *__restric
     constexpr int V = D / 32;
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
+    // launched with programmatic stream serialization: the partials are read only once the
+    // kernel that wrote them (the previous one in the stream) has completed
+    grid_dependency_wait();
     if (row >= rows) return;
     float M = -INFINITY;
     for (int s = lane; s < num_splits; s += 32) M = fmaxf(M, __ldg(lse_part + (size_t)s * rows + row));
@@ -68,21 +71,24 @@ cudaError_t launch_lse_combine(const float *o_part, const float *lse_part, int n
     if (rows <= 0) return cudaSuccess;
     const int threads = 256;
     const int blocks = (int)(((size_t)rows * 32 + threads - 1) / threads);
-    if (out_f32) {
-        if (D == 128)
-            lse_combine_kernel<128, float><<<blocks, threads, 0, stream>>>(
-                o_part, lse_part, num_splits, rows, static_cast<float *>(out), lse);
-        else
-            lse_combine_kernel<64, float><<<blocks, threads, 0, stream>>>(
-                o_part, lse_part, num_splits, rows, static_cast<float *>(out), lse);
-    } else if (D == 128) {
-        lse_combine_kernel<128, __nv_bfloat16><<<blocks, threads, 0, stream>>>(
-            o_part, lse_part, num_splits, rows, static_cast<__nv_bfloat16 *>(out), lse);
-    } else {
-        lse_combine_kernel<64, __nv_bfloat16><<<blocks, threads, 0, stream>>>(
-            o_part, lse_part, num_splits, rows, static_cast<__nv_bfloat16 *>(out), lse);
-    }
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (out_f32)
+        return D == 128 ? cudaLaunchKernelEx(&cfg, lse_combine_kernel<128, float>, o_part, lse_part,
+                                             num_splits, rows, static_cast<float *>(out), lse)
+                        : cudaLaunchKernelEx(&cfg, lse_combine_kernel<64, float>, o_part, lse_part,
+                                             num_splits, rows, static_cast<float *>(out), lse);
+    return D == 128 ? cudaLaunchKernelEx(&cfg, lse_combine_kernel<128, __nv_bfloat16>, o_part, lse_part,
+                                         num_splits, rows, static_cast<__nv_bfloat16 *>(out), lse)
+                    : cudaLaunchKernelEx(&cfg, lse_combine_kernel<64, __nv_bfloat16>, o_part, lse_part,
+                                         num_splits, rows, static_cast<__nv_bfloat16 *>(out), lse);
 }
 
 }  // namespace gqa

@@ -470,6 +470,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const int head_lo = kvh * g + chunk * heads_per_cta;
     const int nh = min(heads_per_cta, g - chunk * heads_per_cta);
     const int P = a.P;
+    // Launched with programmatic stream serialization: the CTA may be resident before the
+    // previous kernel in the stream has finished, and touches no input, output or
+    // workspace byte until it has.  lse_combine behind it may be scheduled from here on.
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     // This split's token range [t0, t1), page aligned (contiguous ranges of
     // ceil(np / num_splits) pages).
@@ -1209,9 +1214,17 @@ cudaError_t launch_t(const DecodeArgs &a, const CUtensorMap &kmap, const CUtenso
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT, FP8, TT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.num_splits, a.Hk * chunks, a.B);
-    decode_kernel<D, NT, FP8, TT><<<grid, kThreads, smem, stream>>>(kmap, vmap, a, hpc, chunks);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_splits, a.Hk * chunks, a.B);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<D, NT, FP8, TT>, kmap, vmap, a, hpc, chunks);
 }
 
 }  // namespace
