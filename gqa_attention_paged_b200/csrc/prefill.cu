@@ -291,8 +291,13 @@ __device__ __forceinline__ void softmax_role(PSmem<D> &sm, const PrefillArgs &a,
 // each is computed on its own, so the outputs do not depend on it.
 __global__ void __launch_bounds__(1024)
     prefill_plan_kernel(const PrefillArgs a, const int T, const int items_per_seq) {
-    __shared__ int hist[kPlanBins];
+    __shared__ __align__(16) int hist[kPlanBins];
     const int total = a.B * items_per_seq;
+    // launched with programmatic stream serialization: the inputs and the plan are touched
+    // only once the previous kernel in the stream (which may still read the plan) is
+    // complete; the prefill CTAs behind this one may become resident from here on
+    grid_dependency_wait();
+    grid_dependents_launch();
     for (int i = threadIdx.x; i < kPlanBins; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     auto cost_of = [&](int idx, int &item) -> int {
@@ -315,26 +320,46 @@ __global__ void __launch_bounds__(1024)
         }
     }
     __syncthreads();
-    // exclusive offsets in descending cost order (warp 0; lane i owns a run of bins)
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        constexpr int per = kPlanBins / 32;
-        int sum = 0;
-        for (int i = 0; i < per; ++i) sum += hist[kPlanBins - 1 - (lane * per + i)];
-        int incl = sum;
+    // exclusive offsets in descending cost order, over the whole block: thread t owns the
+    // four bins 4095 - 4t .. 4092 - 4t (one int4, so a warp reads 32 consecutive vectors),
+    // then a warp scan and a scan of the warp totals
+    static_assert(kPlanBins == 4 * 1024, "four bins per thread of the 1024");
+    {
+        __shared__ int wsum[32];
+        const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+        int4 *h4 = reinterpret_cast<int4 *>(hist);
+        const int4 v = h4[kPlanBins / 4 - 1 - t];  // bins (x, y, z, w) = 4092-4t .. 4095-4t
+        const int s4 = v.x + v.y + v.z + v.w;
+        int incl = s4;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(kAll, incl, o);
-            if (lane >= o) incl += t;
+            const int u = __shfl_up_sync(kAll, incl, o);
+            if (lane >= o) incl += u;
         }
-        int run = incl - sum;
-        for (int i = 0; i < per; ++i) {
-            const int c = kPlanBins - 1 - (lane * per + i);
-            const int h = hist[c];
-            hist[c] = run;
-            run += h;
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = wsum[lane];
+            int wi = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(kAll, wi, o);
+                if (lane >= o) wi += u;
+            }
+            wsum[lane] = wi - w;  // exclusive offset of each warp
+            if (lane == 31) a.plan[0] = wi;
         }
-        if (lane == 31) a.plan[0] = incl;
+        __syncthreads();
+        int run = wsum[warp] + incl - s4;  // bins above this thread's four, in descending order
+        int4 o;
+        o.w = run;
+        run += v.w;
+        o.z = run;
+        run += v.z;
+        o.y = run;
+        run += v.y;
+        o.x = run;
+        h4[kPlanBins / 4 - 1 - t] = o;
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
@@ -357,6 +382,9 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     // the longest items are dispatched first, all heads of an item together
     const int kvh = blockIdx.x % a.Hk;
     const int rank = blockIdx.x / a.Hk;
+    // launched with programmatic stream serialization behind the plan kernel: nothing is
+    // read or written before the plan (and everything before it in the stream) is complete
+    grid_dependency_wait();
     if (rank >= a.plan[0]) return;  // uniform for the whole CTA
     const int item = a.plan[1 + rank];
     const int b = item >> 16, ct = item & 0xffff;
@@ -697,10 +725,21 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &kmap, cons
     if (e != cudaSuccess) return e;
     const int items_per_seq = (a.max_q_len + kQT * T - 1) / (kQT * T);
     if (items_per_seq == 0 || a.B == 0) return cudaSuccess;
-    prefill_plan_kernel<<<1, 1024, 0, stream>>>(a, T, items_per_seq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    prefill_kernel<D><<<a.B * items_per_seq * a.Hk, kThreadsP, smem, stream>>>(kmap, vmap, qmap, a, T);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(1);
+    pc.blockDim = dim3(1024);
+    pc.stream = stream;
+    pc.attrs = attr;
+    pc.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&pc, prefill_plan_kernel, a, T, items_per_seq)) != cudaSuccess) return e;
+    cudaLaunchConfig_t kc = pc;
+    kc.gridDim = dim3(a.B * items_per_seq * a.Hk);
+    kc.blockDim = dim3(kThreadsP);
+    kc.dynamicSmemBytes = smem;
+    return cudaLaunchKernelEx(&kc, prefill_kernel<D>, kmap, vmap, qmap, a, T);
 }
 
 }  // namespace
