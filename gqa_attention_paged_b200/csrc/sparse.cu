@@ -179,6 +179,10 @@ __global__ void __launch_bounds__(kSelThreads) sparse_score_kernel(
     const int g = Hq / Hk;
     const int kvh = blockIdx.y, b = blockIdx.z;
     const int c0 = blockIdx.x * kSelChunk;
+    // launched with programmatic stream serialization: no input or output is touched before
+    // the previous kernel in the stream is complete; the pick kernel may become resident
+    grid_dependency_wait();
+    grid_dependents_launch();
     int L = seq_lens[b];
     if (L < 0 || L > pt_stride * P) L = L < 0 ? 0 : pt_stride * P;  // reported by the pick kernel
     const int np = (L + P - 1) / P;
@@ -253,6 +257,10 @@ __global__ void __launch_bounds__(kSelThreads) sparse_pick_kernel(
     const int kvh = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const size_t row = (size_t)b * Hk + kvh;
+    // behind the score kernel, with programmatic stream serialization: the keys are read
+    // once it is complete; the decode of the chosen pages may become resident
+    grid_dependency_wait();
+    grid_dependents_launch();
     int L = seq_lens[b];
     if (L < 0 || L > pt_stride * P) {
         if (threadIdx.x == 0 && kvh == 0) set_error(err, GQA_ERR_BAD_PAGE);
@@ -394,25 +402,33 @@ cudaError_t launch_sparse_select(const void *q, const void *kt, const int32_t *p
                                  int32_t *sel_pages, uint32_t *keys, int *err,
                                  cudaStream_t stream) {
     if (B == 0) return cudaSuccess;
-    const dim3 sgrid((pt_stride + kSelChunk - 1) / kSelChunk, Hk, B);
-    if (D == 128)
-        sparse_score_kernel<128><<<sgrid, kSelThreads, 0, stream>>>(
-            static_cast<const uint16_t *>(q), static_cast<const uint32_t *>(kt), page_table,
-            pt_stride, seq_lens, Hq, Hk, P, num_pages, topk, window, keys, err);
-    else
-        sparse_score_kernel<64><<<sgrid, kSelThreads, 0, stream>>>(
-            static_cast<const uint16_t *>(q), static_cast<const uint32_t *>(kt), page_table,
-            pt_stride, seq_lens, Hq, Hk, P, num_pages, topk, window, keys, err);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t sc = {};
+    sc.gridDim = dim3((pt_stride + kSelChunk - 1) / kSelChunk, Hk, B);
+    sc.blockDim = dim3(kSelThreads);
+    sc.stream = stream;
+    sc.attrs = attr;
+    sc.numAttrs = 1;
+    const uint16_t *q16 = static_cast<const uint16_t *>(q);
+    const uint32_t *kt32 = static_cast<const uint32_t *>(kt);
+    cudaError_t e = D == 128 ? cudaLaunchKernelEx(&sc, sparse_score_kernel<128>, q16, kt32, page_table, pt_stride,
+                                                  seq_lens, Hq, Hk, P, num_pages, topk, window, keys, err)
+                             : cudaLaunchKernelEx(&sc, sparse_score_kernel<64>, q16, kt32, page_table, pt_stride,
+                                                  seq_lens, Hq, Hk, P, num_pages, topk, window, keys, err);
     if (e != cudaSuccess) return e;
     const size_t smem = sparse_pick_smem_bytes(pt_stride);
     e = cudaFuncSetAttribute(sparse_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    sparse_pick_kernel<<<dim3(Hk, B), kSelThreads, smem, stream>>>(
-        keys, page_table, pt_stride, seq_lens, Hk, P, num_pages, topk, window, sel_table,
-        sel_stride, sel_lens, sel_pages, err);
-    return cudaGetLastError();
+    cudaLaunchConfig_t pc = sc;
+    pc.gridDim = dim3(Hk, B);
+    pc.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&pc, sparse_pick_kernel, static_cast<const uint32_t *>(keys), page_table, pt_stride,
+                           seq_lens, Hk, P, num_pages, topk, window, sel_table, sel_stride, sel_lens,
+                           sel_pages, err);
+    return e;
 }
 
 }  // namespace gqa
