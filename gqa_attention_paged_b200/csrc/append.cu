@@ -34,6 +34,10 @@ __device__ __forceinline__ float block_absmax(float x, float *red) {
 __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     __shared__ float red[2][4];
     const int b = blockIdx.x, kvh = blockIdx.y, d = threadIdx.x;
+    // launched with programmatic stream serialization: nothing is read or written before the
+    // previous kernel in the stream is complete; the decode behind it may become resident
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int L = a.seq_lens[b];
     if (L <= 0) return;  // uniform for the CTA
     if (L > a.pt_stride * a.P) {
@@ -81,8 +85,16 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t stream) {
     if (a.B == 0) return cudaSuccess;
-    append_kernel<<<dim3(a.B, a.Hk), a.D, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B, a.Hk);
+    cfg.blockDim = dim3(a.D);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, append_kernel, a);
 }
 
 }  // namespace gqa
