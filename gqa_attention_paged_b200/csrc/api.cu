@@ -88,11 +88,11 @@ constexpr int kTabUnits = 8, kTabCtx = 5;
 const int kTabUnitsAt[kTabUnits] = {8, 16, 32, 64, 128, 512, 2048, 8192};
 const int kTabCtxAt[kTabCtx] = {512, 2048, 4096, 8192, 32768};
 const unsigned char kBestSplits[2][kTabUnits][kTabCtx] = {
-    {{8, 16, 16, 32, 32}, {8, 16, 16, 16, 16}, {4, 8, 8, 8, 32}, {4, 4, 4, 16, 32}, {2, 2, 8, 16, 16}, {2, 4, 4, 4, 8}, {1, 1, 1, 1, 1}, {1, 1, 1, 1, 1}},
-    {{4, 16, 16, 32, 32}, {8, 8, 16, 16, 16}, {4, 8, 8, 8, 32}, {4, 4, 4, 16, 32}, {2, 2, 8, 16, 16}, {1, 4, 4, 4, 16}, {1, 1, 1, 4, 4}, {1, 1, 1, 1, 1}}};
+    {{8, 16, 16, 32, 32}, {8, 16, 16, 16, 16}, {4, 8, 8, 8, 32}, {4, 4, 4, 16, 32}, {2, 2, 8, 16, 16}, {2, 4, 4, 4, 4}, {1, 1, 1, 1, 1}, {1, 1, 1, 1, 1}},
+    {{8, 16, 16, 16, 32}, {8, 8, 16, 16, 16}, {4, 8, 8, 8, 32}, {4, 4, 4, 16, 32}, {2, 2, 8, 16, 16}, {1, 4, 4, 4, 16}, {1, 1, 1, 4, 4}, {1, 1, 1, 1, 1}}};
 const unsigned char kAutoSplits[2][kTabUnits][kTabCtx] = {
-    {{8, 0, 0, 0, 0}, {8, 0, 0, 16, 0}, {4, 0, 8, 0, 0}, {4, 4, 0, 0, 0}, {2, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}},
-    {{4, 16, 0, 0, 0}, {8, 8, 0, 0, 0}, {4, 8, 8, 0, 0}, {4, 4, 0, 0, 0}, {2, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}}};
+    {{8, 16, 0, 0, 0}, {8, 0, 0, 16, 0}, {4, 8, 8, 0, 0}, {4, 4, 0, 0, 0}, {2, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}},
+    {{8, 16, 0, 0, 0}, {8, 8, 16, 0, 0}, {4, 8, 8, 0, 0}, {4, 4, 0, 0, 0}, {2, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}}};
 
 // Index of the entry of `at` nearest to x in log scale.
 int nearest_log(const int *at, int n, double x) {

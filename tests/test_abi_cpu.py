@@ -197,6 +197,8 @@ def test_measured_split_table():
     assert f(1, 8, 100, 16, 0) == 7          # clamped to ceil(100 / 16) pages
     launches = binding.gqa_paged_decode_kernel_launches
     assert launches(1, 32, 8, 128, 16, 512, 0, 0) == 2    # auto: 8 splits + lse_combine
+    assert launches(1, 32, 8, 128, 16, 2048, 0, 0) == 2   # auto: 16 splits + lse_combine
+    assert launches(4, 32, 8, 128, 16, 2048, 0, 0) == 2   # auto: 8 splits + lse_combine
     assert launches(4, 32, 8, 128, 16, 2048, 1, 0) == 2   # e4m3: 8 splits + lse_combine
     assert launches(64, 32, 8, 128, 16, 2048, 0, 0) == 1  # balanced, in-launch merge
     assert launches(16, 32, 8, 128, 16, 2048, 0, 0) == 2  # balanced, 9 workers per unit: merge kernel
