@@ -838,7 +838,7 @@ def measure_sparse(a, dev, with_cpu):
     # the decode of the chosen pages: B * Hk sequences of one kv head and Hq / Hk heads
     dec_launches = binding.gqa_paged_decode_kernel_launches(
         B * Hk, Hq // Hk, 1, D, P, binding.gqa_paged_sparse_table_stride(pt.shape[1], P, topk, window) * P,
-        0, 0)
+        0, -1)
     cpu = None
     if with_cpu:
         from oracle import oracle
@@ -870,8 +870,8 @@ def measure_sparse(a, dev, with_cpu):
         "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "traffic": traffic_from_profile("sparse70b"),
                      "traffic_key": "sparse70b",
-                     "kernel": "sparse_score_kernel + sparse_pick_kernel + the decode of the chosen pages as "
-                               f"num_splits = 0 schedules it ({dec_launches} launch(es)): the whole call"},
+                     "kernel": "sparse_score_kernel + sparse_pick_kernel + the decode of the chosen pages on "
+                               f"the balanced schedule ({dec_launches} launch(es)): the whole call"},
         "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hin),
                 "d2h_bytes_per_step": sum(p_[0].numel() * p_[0].element_size() for p_ in hout),

@@ -659,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 // Flat tile space: sequence b owns tiles [U*pre[b], U*pre[b+1]) with pre[] the prefix of
 // nt_b = ceil(L_b / 16) and U = Hk * head chunks units per sequence; unit y of sequence
 // b owns [U*pre[b] + y*nt_b, ... + nt_b).  With T tiles and NW workers (sk_workers: at most
-// one per kMinTilesPerWorker tiles, or per kMinTilesPerWorkerSmall for small launches),
-// worker W owns [W*T/NW, (W+1)*T/NW) (floor divisions): every worker gets one tile more or
+// one per kMinTilesPerWorker tiles, or per kMinTilesPerWorkerSmall for small launches,
+// and a multiple of the unit count where the units merge in the launch), worker W owns [W*T/NW, (W+1)*T/NW) (floor divisions): every worker gets one tile more or
 // less than any other.
 //
 // Each consumer warp is one worker with a private sub-ring of S/4 stages fed by its own
@@ -673,13 +673,22 @@ constexpr int kMinTilesPerWorker = 16;  // 16-token tiles; half as many 32-token
 // streams are latency-bound, so more of them in flight finish sooner.
 constexpr int kMinTilesPerWorkerSmall = 4;
 
-// Workers of a launch with T tiles of TT tokens and `workers` consumer warps.
+// Workers of a launch with T tiles of TT tokens, `workers` consumer warps and `units`
+// (sequence, kv head, head chunk) units.  Where the units merge in the launch (fewer than
+// kDeferMinWorkersPerUnit workers each), the count is rounded down to a multiple of the
+// units if that keeps three quarters of the workers: with units of equal length every
+// worker then holds one piece of one unit instead of the end of one and the start of the
+// next, so it writes one piece, and each unit merges c pieces that finish together.
+// Measured (B=20..64 at ctx 2048, bf16 and e4m3): 3-7% faster, no slower elsewhere.
 template <int TT>
-__device__ __forceinline__ long long sk_workers(long long T, long long workers) {
+__device__ __forceinline__ long long sk_workers(long long T, long long workers, long long units) {
     constexpr long long kMin = kMinTilesPerWorker * 16 / TT;
     const long long nw = T / kMin;
     const long long per = nw * 4 < workers ? kMinTilesPerWorkerSmall : kMin;
-    return min(workers, max(1LL, T / per));
+    const long long r = min(workers, max(1LL, T / per));
+    const long long c = units > 0 ? r / units : 0;
+    if (c >= 1 && c < kDeferMinWorkersPerUnit && 4 * c * units >= 3 * r) return c * units;
+    return r;
 }
 // Launches whose units average more than kDeferMinWorkersPerUnit workers each leave their
 // pieces to a second kernel (piece_merge_kernel, the DEFER instance), which merges every
@@ -859,7 +868,7 @@ __global__ void __launch_bounds__(balanced_threads<FP8>(), kStreamCtasPerSm)
     __syncthreads();
 
     const long long T = (long long)U * pre[B];
-    const long long NW = sk_workers<TT>(T, (long long)gridDim.x * kConsumerWarps);
+    const long long NW = sk_workers<TT>(T, (long long)gridDim.x * kConsumerWarps, (long long)B * U);
     const long long W0cta = (long long)blockIdx.x * kConsumerWarps;
 
     // Sequences with no tokens have no tiles: their outputs are written here (zeros, -inf).
@@ -1110,7 +1119,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
     if (warp == 0) tile_prefix<TT>(a, pre_m, a.pt_stride * a.P, nullptr, lane);
     __syncthreads();
     const long long T = (long long)U * pre_m[a.B];
-    const long long NW = sk_workers<TT>(T, (long long)a.grid * kConsumerWarps);
+    const long long NW = sk_workers<TT>(T, (long long)a.grid * kConsumerWarps, (long long)a.B * U);
     const int slot_floats = (heads_per_cta * (D + 1) + 3) & ~3;
     for (long long u = blockIdx.x; u < (long long)a.B * U; u += gridDim.x) {
         const int b = (int)(u / U), y = (int)(u % U);

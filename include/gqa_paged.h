@@ -421,7 +421,9 @@ size_t gqa_paged_sparse_decode_workspace_size(int B, int Hq, int Hk, int head_di
 /*
  * Sparse decode: the selection, then the decode over the chosen pages, on `stream`.
  * q, pools, page_table, seq_lens, scale, num_splits, out, lse as for gqa_paged_decode()
- * (bf16 pools); kt as for gqa_paged_kt_build(); B * Hk <= 65535.  The workspace holds the
+ * (bf16 pools), except that num_splits = 0 runs the balanced schedule for the decode of the
+ * chosen pages (measured faster on the 70B shape than the split count the decode table
+ * gives for that size); kt as for gqa_paged_kt_build(); B * Hk <= 65535.  The workspace holds the
  * chosen-page table between the two kernels; zero it once before first use.
  */
 int gqa_paged_sparse_decode(const void *q, const void *k_pages, const void *v_pages,

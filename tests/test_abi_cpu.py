@@ -214,3 +214,17 @@ def test_measured_split_table():
     assert ws(8, 32, 8, 128, 16, 4096, 0, 0) == ws(8, 32, 8, 128, 16, 4096, 0, -1)
     assert ws(8, 32, 8, 128, 16, 4096, 0, 0) != ws(8, 32, 8, 128, 16, 4096, 0, 4)
     assert ws(1, 32, 8, 128, 16, 512, 0, 0) == 256 + (8 * 32 * 128 * 4 + 255) // 256 * 256 + 1024
+
+
+def test_sparse_decode_runs_the_balanced_schedule_by_default():
+    """num_splits = 0 in the sparse decode means the balanced schedule for the decode of the
+    chosen pages (its workspace is the balanced one, not that of the split count the dense
+    table gives for 32 one-kv-head sequences of ~2K tokens)."""
+    lib = binding.load()
+    f = lib.gqa_paged_sparse_decode_workspace_size
+    args = (4, 64, 8, 128, 64, 512, 32, 32)
+    assert f(*args, 0) == f(*args, -1)
+    assert f(*args, 0) != f(*args, 8)
+    ss = lib.gqa_paged_sparse_table_stride(512, 64, 32, 32)
+    dec = lib.gqa_paged_decode_workspace_size
+    assert dec(32, 8, 1, 128, 64, ss * 64, 0, -1) != dec(32, 8, 1, 128, 64, ss * 64, 0, 0)

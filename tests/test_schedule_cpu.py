@@ -3,7 +3,8 @@ partition among workers, the owner of a tile, and the merge pieces of units that
 share.  The formulas are the ones decode_sk_kernel evaluates (restated here): worker W
 owns flat tiles [W*T//NW, (W+1)*T//NW) with NW = min(workers, max(1, T // per)), per = 16
 tiles of 16 tokens (8 of 32 tokens), or 4 when T // per workers would be under a quarter of
-them; the owner
+them, then rounded down to a multiple c of the unit count when 1 <= c < 8 (units that merge
+in the launch) and that keeps three quarters of NW; the owner
 of tile t is ((t+1)*NW + T-1)//T - 1;
 a unit cut between workers leaves one piece per worker, side 1 for the worker where the
 unit begins and side 0 for the others.  The last piece of a unit merges them in the same
@@ -15,10 +16,14 @@ import random
 import pytest
 
 
-def n_workers(workers, T, tile_tokens=16):
+def n_workers(workers, T, tile_tokens=16, units=0):
     base = 16 * 16 // tile_tokens
     per = 4 if (T // base) * 4 < workers else base
-    return min(workers, max(1, T // per))
+    r = min(workers, max(1, T // per))
+    c = r // units if units > 0 else 0
+    if 1 <= c < 8 and 4 * c * units >= 3 * r:
+        return c * units
+    return r
 
 
 def start(W, T, NW):
@@ -35,7 +40,7 @@ def schedule(tiles_per_seq, U, workers):
     for n in tiles_per_seq:
         pre.append(pre[-1] + n)
     T = U * pre[-1]
-    NW = n_workers(workers, T)
+    NW = n_workers(workers, T, units=len(tiles_per_seq) * U)
     finals, pieces, slots = {}, {}, {}
     for W in range(workers):
         s, e = start(W, T, NW), start(W + 1, T, NW)
@@ -105,6 +110,40 @@ def test_units_are_written_exactly_once():
                 assert got == want, (tiles, U, workers, key)
 
 
+@pytest.mark.parametrize("B,U,ntiles,workers", [(20, 8, 128, 1184), (32, 8, 128, 1184),
+                                                (32, 8, 64, 1184), (64, 8, 128, 1184),
+                                                (128, 8, 128, 1184), (3, 5, 17, 40)])
+def test_unit_aligned_worker_count(B, U, ntiles, workers):
+    """Units of equal length that merge in the launch: the worker count is a multiple c of
+    the units, every unit is cut into exactly c pieces (or held whole when c = 1), and no
+    worker holds parts of two units."""
+    units = B * U
+    T = units * ntiles
+    NW = n_workers(workers, T, 16, units)
+    r = n_workers(workers, T)
+    c = NW // units
+    assert NW % units == 0 and 1 <= c < 8 and 4 * NW >= 3 * r
+    _, NW2, finals, pieces = schedule([ntiles] * B, U, workers)
+    assert NW2 == NW
+    if c == 1:
+        assert not pieces and all(len(v) == 1 for v in finals.values()) and len(finals) == units
+    else:
+        assert not finals and all(len(v) == c for v in pieces.values()) and len(pieces) == units
+        held = [W for v in pieces.values() for W, _ in v]
+        assert len(held) == len(set(held)) == NW
+
+
+def test_worker_count_unaligned_outside_the_in_launch_merge():
+    # 11.84 workers per unit: the merge kernel's launch keeps the plain count
+    assert n_workers(1184, 100 * 200, units=100) == n_workers(1184, 100 * 200) == 1184
+    # B=16 at ctx 2048: 16 tiles per worker already give 8 per unit
+    assert n_workers(1184, 128 * 128, units=128) == 1024
+    # rounding would drop more than a quarter (640 units: c = 1 keeps 54%)
+    assert n_workers(1184, 640 * 128, units=640) == 1184
+    # a few long units (small launch, 32 per unit): unchanged
+    assert n_workers(1184, 8 * 128, units=8) == n_workers(1184, 8 * 128) == 256
+
+
 def test_slot_indices_stay_in_the_workspace():
     """Slots W*2+side < 2 * (SMs * CTAs per SM * 4 workers), the bound the workspace is
     sized for; counters b*U+y < B*Hq."""
@@ -138,7 +177,7 @@ def merge_kernel_reads(tiles_per_seq, U, workers):
     for n in tiles_per_seq:
         pre.append(pre[-1] + n)
     T = U * pre[-1]
-    NW = n_workers(workers, T)
+    NW = n_workers(workers, T, units=len(tiles_per_seq) * U)
     reads = {}
     for b, n in enumerate(tiles_per_seq):
         if n == 0:
