@@ -107,6 +107,14 @@ __device__ __forceinline__ void consumer_bar() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
+// Adds `bytes` to the barrier's expected transaction count without an arrival (the
+// producer arrives later, once it has also written the stage's scales).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ int clamp_len(int L, int Lmax, int *err) {
     if (L < 0 || L > Lmax) {
         set_error(err, GQA_ERR_BAD_PAGE);
@@ -925,15 +933,14 @@ __global__ void __launch_bounds__(balanced_threads<FP8>(), kStreamCtasPerSm)
                 set_error(a.err, GQA_ERR_BAD_PAGE);
                 mbar_arrive(&sm.full[stage]);  // no copy: the tile computes on stale data
             } else {
-                if (FP8) {
-                    sm.kscale[stage][0] = __ldg(a.k_scale + (size_t)phys * a.Hk + kvh);
-                    sm.vscale[stage][0] = __ldg(a.v_scale + (size_t)phys * a.Hk + kvh);
-                    sm.kscale[stage][1] = second ? __ldg(a.k_scale + (size_t)phys2 * a.Hk + kvh) : sm.kscale[stage][0];
-                    sm.vscale[stage][1] = second ? __ldg(a.v_scale + (size_t)phys2 * a.Hk + kvh) : sm.vscale[stage][0];
-                }
+                // e4m3: the copies are issued first (expected bytes, no arrival), the scales are
+                // loaded while they fly, and the producer's arrival after the scales' stores
+                // releases both.  Loading the scales first put a second dependent round trip
+                // (page-table entry, then scales) before every copy.
                 const int row = (phys * a.Hk + kvh) * P + tok0 % P;
                 if (!two) {
-                    mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
+                    if (FP8) mbar_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
+                    else mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kTileBytes);
 #pragma unroll
                     for (int bx = 0; bx < C::kBoxes; ++bx) {
                         tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128, &kmap, &sm.full[stage],
@@ -944,7 +951,8 @@ __global__ void __launch_bounds__(balanced_threads<FP8>(), kStreamCtasPerSm)
                 } else {
                     // P-row boxes; rows past the first page are the second page's
                     const int row2 = (phys2 * a.Hk + kvh) * P;
-                    mbar_arrive_expect_tx(&sm.full[stage], (second ? 2 : 1) * 2 * C::kBoxes * P * 128);
+                    if (FP8) mbar_expect_tx(&sm.full[stage], (second ? 2 : 1) * 2 * C::kBoxes * P * 128);
+                    else mbar_arrive_expect_tx(&sm.full[stage], (second ? 2 : 1) * 2 * C::kBoxes * P * 128);
 #pragma unroll
                     for (int bx = 0; bx < C::kBoxes; ++bx) {
                         tma_load_2d(sm.tiles[stage][0] + bx * kTile * 128, &kmap, &sm.full[stage],
@@ -958,6 +966,13 @@ __global__ void __launch_bounds__(balanced_threads<FP8>(), kStreamCtasPerSm)
                                         &sm.full[stage], bx * C::kBoxCols, row2, pol);
                         }
                     }
+                }
+                if (FP8) {
+                    sm.kscale[stage][0] = __ldg(a.k_scale + (size_t)phys * a.Hk + kvh);
+                    sm.vscale[stage][0] = __ldg(a.v_scale + (size_t)phys * a.Hk + kvh);
+                    sm.kscale[stage][1] = second ? __ldg(a.k_scale + (size_t)phys2 * a.Hk + kvh) : sm.kscale[stage][0];
+                    sm.vscale[stage][1] = second ? __ldg(a.v_scale + (size_t)phys2 * a.Hk + kvh) : sm.vscale[stage][0];
+                    mbar_arrive(&sm.full[stage]);
                 }
             }
             issued = r + 1;
