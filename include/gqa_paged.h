@@ -128,7 +128,8 @@ int gqa_pick_splits(int B, int Hk, int max_seq_len, int page_size, int kv_dtype)
  *   num_splits 0 = automatic: for B <= 2048 a balanced persistent schedule: all
  *              (sequence, kv head) tiles of 16 tokens are laid end to end and shared
  *              equally by the workers of a fixed grid, and units cut between workers are
- *              merged by log-sum-exp inside the same launch -- except for the small
+ *              merged by log-sum-exp inside the same launch (by a second kernel where the
+ *              units average more than 8 workers each) -- except for the small
  *              problems (a few sequences of short context pt_stride*page_size) where the
  *              split schedule measured faster, which run splits with the measured count;
  *              for larger B, splits with the count gqa_pick_splits gives.
