@@ -201,7 +201,7 @@ def test_measured_split_table():
     assert launches(4, 32, 8, 128, 16, 2048, 0, 0) == 2   # auto: 8 splits + lse_combine
     assert launches(4, 32, 8, 128, 16, 2048, 1, 0) == 2   # e4m3: 8 splits + lse_combine
     assert launches(64, 32, 8, 128, 16, 2048, 0, 0) == 1  # balanced, in-launch merge
-    assert launches(16, 32, 8, 128, 16, 2048, 0, 0) == 2  # balanced, 9 workers per unit: merge kernel
+    assert launches(16, 32, 8, 128, 16, 2048, 0, 0) == 2  # balanced, 9.25 grid workers per unit: merge kernel
     assert launches(32, 32, 8, 128, 16, 2048, 0, 0) == 1  # balanced, in-launch merge
     assert launches(16, 32, 8, 128, 16, 512, 0, -1) == 2  # balanced on request, merge kernel
     assert launches(32, 32, 8, 128, 16, 512, 0, -1) == 1  # balanced on request, in-launch merge

@@ -215,7 +215,7 @@ def test_defer_policy_on_the_named_shapes():
     assert defers(4, 64, 8, True, grid)        # 70B long context: 32 units, 37 workers each
     assert defers(1, 32, 8, True, grid)        # one sequence
     assert not defers(64, 32, 8, True, grid)   # B=64 sweep: 2 workers per unit
-    assert defers(16, 32, 8, True, grid)       # 7B-shaped batch: 9 workers per unit
+    assert defers(16, 32, 8, True, grid)       # 7B-shaped batch: 9.25 grid workers per unit
     assert not defers(32, 32, 8, True, grid)   # 4.6 workers per unit
     assert not defers(8, 32, 8, False, grid)   # PackGQA off: one unit per head
     assert defers(64, 32, 2, True, grid)       # groups of 16: always the merge kernel
